@@ -1,0 +1,221 @@
+"""R-SWA CPU oracle (FP64) -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its binding in ``ring_sliding_window_b200``) never imports, links or executes
+anything here, and this package imports nothing from it.
+
+The arithmetic lives in ``oracle.c`` (plain C, double precision); this module
+only marshals numpy arrays through ctypes and keeps per-(layer, sequence) ring
+objects for multi-layer, multi-sequence runs.
+
+Method source, by page title and section:
+  "开源5天Star破万之后：百度Unlimited-OCR的爆火路径复盘", §2.1 (ring
+  sliding-window attention: prefill kept whole, warm-up append, steady-state
+  ring overwrite of slot prefill_len + ring_pos) and §2.3 (no-repeat n-gram ban
+  restricted to a sliding window).
+
+Pins (in tests/): float64 SDPA from torch, closed forms, brute force over the
+union key set, the transformers no-repeat-ngram processor, hand-built n-gram
+fixtures under tests/golden/.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+ORC_OK, ORC_EINVAL, ORC_ENOMEM, ORC_ESTATE, ORC_EDATA = 0, 1, 2, 4, 6
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (OpenMP when available)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + ".tmp"
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_fp = ctypes.POINTER(ctypes.c_float)
+_ip = ctypes.POINTER(ctypes.c_int32)
+_lp = ctypes.POINTER(ctypes.c_int64)
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    # ORACLE_LIB_OVERRIDE points the pins at a deliberately broken build of
+    # oracle.c (tests/test_oracle_mutants.py), to show that they catch it.
+    lib = ctypes.CDLL(os.environ.get("ORACLE_LIB_OVERRIDE") or build())
+    lib.oracle_attend.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                  ctypes.c_double, _dp]
+    lib.oracle_attend.restype = ctypes.c_int
+    lib.oracle_prefill.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_double, ctypes.c_int64, ctypes.c_int64, _dp]
+    lib.oracle_prefill.restype = ctypes.c_int
+    lib.oracle_ring_create.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
+    lib.oracle_ring_create.restype = ctypes.c_void_p
+    lib.oracle_ring_destroy.argtypes = [ctypes.c_void_p]
+    lib.oracle_ring_destroy.restype = None
+    lib.oracle_ring_prefill.argtypes = [ctypes.c_void_p, _dp, _dp]
+    lib.oracle_ring_prefill.restype = ctypes.c_int
+    lib.oracle_ring_step.argtypes = [ctypes.c_void_p, _dp, _dp, _dp, ctypes.c_double, _dp, _lp, _lp]
+    lib.oracle_ring_step.restype = ctypes.c_int
+    lib.oracle_ring_snapshot.argtypes = [ctypes.c_void_p, _dp, _dp]
+    lib.oracle_ring_snapshot.restype = ctypes.c_int64
+    lib.oracle_ring_ring_pos.argtypes = [ctypes.c_void_p]
+    lib.oracle_ring_ring_pos.restype = ctypes.c_int64
+    lib.oracle_ring_len.argtypes = [ctypes.c_void_p]
+    lib.oracle_ring_len.restype = ctypes.c_int64
+    lib.oracle_ngram_ban.argtypes = [_fp, ctypes.c_int64, _ip, ctypes.c_int64, _ip, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.oracle_ngram_ban.restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, t):
+    return a.ctypes.data_as(t)
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def attend(q, k, v, scale: float) -> np.ndarray:
+    """Softmax attention of one query q[d] over keys k[n, d] and values v[n, d]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    n, d = k.shape
+    out = np.empty(d, dtype=np.float64)
+    rc = _load().oracle_attend(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), n, d, d, float(scale),
+                               _ptr(out, _dp))
+    if rc != ORC_OK:
+        raise ValueError(f"oracle_attend failed ({rc})")
+    return out
+
+
+def prefill(q, k, v, scale: float, row_lo: int = 0, row_hi: int | None = None) -> np.ndarray:
+    """Causal prefill attention of one sequence; q, k, v: [P, H, d].
+
+    Returns out[P, H, d]; rows outside [row_lo, row_hi) are left as NaN.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    P, H, d = q.shape
+    row_hi = P if row_hi is None else row_hi
+    out = np.full((P, H, d), np.nan, dtype=np.float64)
+    rc = _load().oracle_prefill(_ptr(q, _dp), _ptr(k, _dp), _ptr(v, _dp), P, H, d, float(scale),
+                                row_lo, row_hi, _ptr(out, _dp))
+    if rc != ORC_OK:
+        raise ValueError(f"oracle_prefill failed ({rc})")
+    return out
+
+
+class Ring:
+    """One (layer, sequence) R-SWA cache simulated by the oracle."""
+
+    def __init__(self, prefill_len: int, window: int, heads: int, head_dim: int):
+        lib = _load()
+        self._h = lib.oracle_ring_create(prefill_len, window, heads, head_dim)
+        if not self._h:
+            raise ValueError("oracle_ring_create failed")
+        self.P, self.W, self.H, self.d = prefill_len, window, heads, head_dim
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h and _lib is not None:
+            _lib.oracle_ring_destroy(h)
+
+    def prefill(self, k, v) -> None:
+        k = _f64(k).reshape(self.P, self.H, self.d)
+        v = _f64(v).reshape(self.P, self.H, self.d)
+        rc = _lib.oracle_ring_prefill(self._h, _ptr(k, _dp), _ptr(v, _dp))
+        if rc != ORC_OK:
+            raise ValueError(f"oracle_ring_prefill failed ({rc})")
+
+    def step(self, q, k_new, v_new, scale: float):
+        """Write one generated token and attend.  Returns (out[H, d], slot, len)."""
+        q = _f64(q).reshape(self.H, self.d)
+        k_new = _f64(k_new).reshape(self.H, self.d)
+        v_new = _f64(v_new).reshape(self.H, self.d)
+        out = np.empty((self.H, self.d), dtype=np.float64)
+        slot = ctypes.c_int64(-1)
+        n = ctypes.c_int64(-1)
+        rc = _lib.oracle_ring_step(self._h, _ptr(q, _dp), _ptr(k_new, _dp), _ptr(v_new, _dp),
+                                   float(scale), _ptr(out, _dp), ctypes.byref(slot), ctypes.byref(n))
+        if rc != ORC_OK:
+            raise ValueError(f"oracle_ring_step failed ({rc})")
+        return out, int(slot.value), int(n.value)
+
+    def snapshot(self):
+        """(k[P+W, H, d], v[P+W, H, d], entries held)."""
+        shape = (self.P + self.W, self.H, self.d)
+        k = np.empty(shape, dtype=np.float64)
+        v = np.empty(shape, dtype=np.float64)
+        n = _lib.oracle_ring_snapshot(self._h, _ptr(k, _dp), _ptr(v, _dp))
+        return k, v, int(n)
+
+    @property
+    def ring_pos(self) -> int:
+        return int(_lib.oracle_ring_ring_pos(self._h))
+
+    @property
+    def length(self) -> int:
+        return int(_lib.oracle_ring_len(self._h))
+
+
+def ngram_ban(logits: np.ndarray, history: np.ndarray, hist_len, n: int, window: int) -> int:
+    """Apply the windowed no-repeat n-gram ban in place.
+
+    logits: float32 [rows, vocab] (C-contiguous), history: int32 [rows, >=window],
+    hist_len: int32 [rows] or None (every row holds `window` tokens).
+    Returns 0, or minus the number of rows rejected as bad data (left untouched).
+    """
+    if logits.dtype != np.float32 or not logits.flags.c_contiguous:
+        raise TypeError("logits must be C-contiguous float32")
+    history = np.ascontiguousarray(history, dtype=np.int32)
+    rows, vocab = logits.shape
+    hl = None if hist_len is None else np.ascontiguousarray(hist_len, dtype=np.int32)
+    rc = _load().oracle_ngram_ban(
+        _ptr(logits, _fp), vocab, _ptr(history, _ip), history.shape[1] if rows else window,
+        None if hl is None else _ptr(hl, _ip), rows, vocab, n, window)
+    if rc > 0:
+        raise ValueError(f"oracle_ngram_ban rejected its arguments ({rc})")
+    return int(rc)
+
+
+class RingModel:
+    """Oracle state for a whole batch: one Ring per (layer, sequence)."""
+
+    def __init__(self, prefill_lens, window: int, layers: int, heads: int, head_dim: int):
+        self.P = [int(p) for p in prefill_lens]
+        self.W, self.L, self.H, self.d = window, layers, heads, head_dim
+        self.rings = [[Ring(p, window, heads, head_dim) for p in self.P] for _ in range(layers)]
+
+    def prefill(self, layer: int, b: int, k, v) -> None:
+        self.rings[layer][b].prefill(k, v)
+
+    def step(self, layer: int, q, k_new, v_new, scale: float) -> np.ndarray:
+        """q, k_new, v_new: [B, H, d] for one layer; returns out[B, H, d]."""
+        outs = [self.rings[layer][b].step(q[b], k_new[b], v_new[b], scale)[0]
+                for b in range(len(self.P))]
+        return np.stack(outs)
