@@ -1,0 +1,536 @@
+#!/usr/bin/env python
+"""R-SWA decode benchmark on B200: decode steps/s, KV-read GB/s vs HBM, prefill TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--also NAMES|none] [--cpu-seconds S]
+
+A timed step is one generated token of the whole batch: for every layer the
+fused ring write + split-K attention + combine (rswa_decode_step), then the
+ring advance and the windowed n-gram ban over the batch's logits -- one CUDA
+graph replay.  The prefill (cache fill + causal attention) is a once-per-batch
+phase; it is timed in the same run and reported under "prefill".
+
+Timing: CUDA events on the launching stream, L2 flushed (256 MiB write)
+before every timed step, outside the events; with N > 1 GPUs every rank runs
+its own replica of the workload (weak scaling) and the time is the max over
+ranks.  rank 0 prints one JSON line.
+
+--impl reference times the FP64 CPU oracle (the only other implementation of
+the method: the pages publish no code) on the host cores, on a bounded
+sample of the same workload, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from ring_sliding_window_b200 import synth  # noqa: E402
+
+METRIC = "R-SWA decode steps/s and KV-read GB/s vs HBM peak; prefill TFLOP/s (1xB200)"
+UNIT = "decode steps/s"
+DATASHEET_HBM_GBS = 8000.0
+DATASHEET_BF16_TFLOPS = 2250.0
+FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"unavailable": "nvidia-smi not runnable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"unavailable": "no samples"}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def kv_bytes_per_layer(w: synth.Workload, t_list):
+    """Algorithmic bytes of one rswa_decode_step (one layer): K and V rows of
+    every valid slot, q, k_new/v_new read, ring write, output write."""
+    e = w.elem_bytes
+    row = w.heads * w.head_dim * e
+    total = 0
+    for b, P in enumerate(w.prefill_lens):
+        t = t_list[b]
+        total += 2 * (P + min(t + 1, w.window)) * row + row + 2 * row + 2 * row + row
+    return total
+
+
+def prefill_flops_per_layer(w: synth.Workload):
+    return sum(4 * w.heads * w.head_dim * P * (P + 1) // 2 for P in w.prefill_lens)
+
+
+# --------------------------------------------------------------------------
+class DecodeRig:
+    """State, graph-captured token step and its I/O buffers for one workload."""
+
+    def __init__(self, w: synth.Workload, start_t: int, fill: str, stream: torch.cuda.Stream):
+        from ring_sliding_window_b200 import rswa
+        self.w, self.s = w, stream
+        L, B, H, d = w.layers, w.batch, w.heads, w.head_dim
+        ng = None if fill == "prefill" else [start_t] * B
+        if w.n_generated is not None and fill != "prefill":
+            ng = list(w.n_generated)
+        self.st = rswa.State(B, L, H, d, w.window, w.prefill_lens, dtype=w.dtype, n_generated=ng)
+        self.q = torch.empty(L, B, H, d, dtype=w.dtype, device="cuda")
+        self.kn = torch.empty_like(self.q)
+        self.vn = torch.empty_like(self.q)
+        self.out = torch.empty_like(self.q)
+        for l in range(L):
+            a, b_, c = synth.decode_qkv(w, l, 0, "cuda")
+            self.q[l].copy_(a)
+            self.kn[l].copy_(b_)
+            self.vn[l].copy_(c)
+        rows = B
+        logits, hist, _ = synth.ngram_inputs(rows, synth.VOCAB, synth.NGRAM_SIZE, synth.NGRAM_WINDOW,
+                                             synth.seed(w.cfg_id, 0, 800_000))
+        self.logits = logits.cuda()
+        self.hist = hist.cuda()
+        self.prefill_ms = None
+        if fill == "random":
+            for l in range(L):
+                g = torch.Generator(device="cuda").manual_seed(synth.seed(w.cfg_id, l, 900_000))
+                self.st.k_cache[l].normal_(generator=g)
+                self.st.v_cache[l].normal_(generator=g)
+        self.graph = None
+
+    def prefill_all(self, flush, time_it=True):
+        """Run rswa_prefill on every layer; returns per-layer event times (ms)."""
+        w = self.w
+        q, k, v = synth.prefill_qkv(w, 0, "cuda")
+        out = torch.empty_like(q)
+        times = []
+        with torch.cuda.stream(self.s):
+            for l in range(w.layers):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(self.s)
+                self.st.prefill(l, q, k, v, out, stream=self.s)
+                e1.record(self.s)
+                times.append((e0, e1))
+        self.s.synchronize()
+        return [a.elapsed_time(b) for a, b in times]
+
+    def token(self):
+        from ring_sliding_window_b200 import rswa
+        w = self.w
+        for l in range(w.layers):
+            self.st.decode_step(l, self.q[l], self.kn[l], self.vn[l], self.out[l], stream=self.s)
+        self.st.advance(stream=self.s)
+        rswa.rswa_ngram_mask(self.logits, self.hist, None, synth.NGRAM_SIZE, synth.NGRAM_WINDOW,
+                             stream=self.s)
+
+    def capture(self):
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.s):
+            self.token()
+        torch.cuda.synchronize()
+
+    def launches_per_token(self):
+        return 2 * self.w.layers + 2
+
+    def ring_t(self):
+        n, _, _ = self.st.ring(stream=self.s)
+        return n
+
+
+def _barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def timed_tokens(rig: DecodeRig, steps: int, warmup: int, flush, sampler=None):
+    """Replay the token graph; returns (per-step ms list, per-step t lists)."""
+    s = rig.s
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            flush.zero_()
+            rig.graph.replay()
+    s.synchronize()
+    t0 = rig.ring_t()
+    _barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    if sampler:
+        sampler.start()
+    with torch.cuda.stream(s):
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(s)
+            rig.graph.replay()
+            evs[i][1].record(s)
+    s.synchronize()
+    _barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = [a.elapsed_time(b) for a, b in evs]
+    ts = [[t + i for t in t0] for i in range(steps)]
+    return ms, ts, clocks
+
+
+def timed_decode_launches(rig: DecodeRig, n: int, flush):
+    """Eager rswa_decode_step launches (split-K + combine), each bracketed by
+    events after an L2 flush that keeps the GPU busy while the CPU enqueues."""
+    w, s = rig.w, rig.s
+    evs = []
+    t0 = rig.ring_t()
+    with torch.cuda.stream(s):
+        for i in range(n):
+            l = i % w.layers
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            rig.st.decode_step(l, rig.q[l], rig.kn[l], rig.vn[l], rig.out[l], stream=s)
+            e1.record(s)
+            evs.append((e0, e1))
+    s.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return ms, t0
+
+
+def e2e_tokens(rig: DecodeRig, steps: int, warmup: int, flush):
+    """Token steps through the public API with host buffers: pinned H2D of the
+    step's q/k_new/v_new (all layers), logits and history; D2H of all layers'
+    outputs and the masked logits; all inside the timed region."""
+    s = rig.s
+    hq = torch.empty(rig.q.shape, dtype=rig.q.dtype, pin_memory=True)
+    hk, hv = torch.empty_like(hq, pin_memory=True), torch.empty_like(hq, pin_memory=True)
+    hq.copy_(rig.q.cpu()); hk.copy_(rig.kn.cpu()); hv.copy_(rig.vn.cpu())
+    hl = rig.logits.cpu().pin_memory()
+    hh = rig.hist.cpu().pin_memory()
+    ho = torch.empty_like(hq, pin_memory=True)
+    hlo = torch.empty_like(hl, pin_memory=True)
+    h2d = 3 * hq.numel() * hq.element_size() + hl.numel() * 4 + hh.numel() * 4
+    d2h = ho.numel() * ho.element_size() + hlo.numel() * 4
+
+    def one():
+        rig.q.copy_(hq, non_blocking=True)
+        rig.kn.copy_(hk, non_blocking=True)
+        rig.vn.copy_(hv, non_blocking=True)
+        rig.logits.copy_(hl, non_blocking=True)
+        rig.hist.copy_(hh, non_blocking=True)
+        rig.graph.replay()
+        ho.copy_(rig.out, non_blocking=True)
+        hlo.copy_(rig.logits, non_blocking=True)
+
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            flush.zero_()
+            one()
+    s.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    _barrier()
+    with torch.cuda.stream(s):
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(s)
+            one()
+            evs[i][1].record(s)
+    s.synchronize()
+    _barrier()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return ms, h2d, d2h
+
+
+# --------------------------------------------------------------------------
+def cpu_oracle_rate(w: synth.Workload, seconds: float, max_steps=None, layers_per_step=None):
+    """The oracle as it stands, on this host's cores: decode steps (all layers of
+    the batch, plus the n-gram ban) from t = 0 until `seconds` have passed."""
+    import numpy as np
+
+    import oracle
+    L = w.layers if layers_per_step is None else layers_per_step
+    rng = np.random.default_rng(0)
+    model = oracle.RingModel(w.prefill_lens, w.window, L, w.heads, w.head_dim)
+    for l in range(L):
+        for b, P in enumerate(w.prefill_lens):
+            model.prefill(l, b, rng.standard_normal((P, w.heads, w.head_dim)),
+                          rng.standard_normal((P, w.heads, w.head_dim)))
+    qkv = [rng.standard_normal((3, w.batch, w.heads, w.head_dim)) for _ in range(L)]
+    logits, hist, _ = synth.ngram_inputs(w.batch, synth.VOCAB, synth.NGRAM_SIZE, synth.NGRAM_WINDOW, 1)
+    lg, hi = logits.numpy(), hist.numpy()
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        for l in range(L):
+            model.step(l, qkv[l][0], qkv[l][1], qkv[l][2], w.scale)
+        oracle.ngram_ban(lg, hi, None, synth.NGRAM_SIZE, synth.NGRAM_WINDOW)
+        steps += 1
+        el = time.perf_counter() - t0
+        if (el >= seconds and steps >= 2) or (max_steps and steps >= max_steps):
+            break
+    rate = steps / el * (L / w.layers)  # full-model decode steps per second
+    return rate, steps, el, oracle.num_threads(), L
+
+
+# --------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    hbm_peak, tc_peak, peak_src = measured_peaks()
+    w = synth.workload(args.workload)
+    dev = torch.cuda.current_device()
+    s = torch.cuda.Stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    # ---- prefill (fills the caches of the main workload), then decode from t = 0
+    rig = DecodeRig(w, 0, "prefill", s)
+    pf_ms = rig.prefill_all(flush)
+    rig.capture()
+    sampler = ClockSampler(dev if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dev]))
+    ms, ts, clocks = timed_tokens(rig, args.steps, args.warmup, flush, sampler)
+    total_ms = sum(ms)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    value = world * args.steps / (total_ms / 1e3)
+    kv_bytes = sum(w.layers * kv_bytes_per_layer(w, t) for t in ts)
+    kv_gbs = kv_bytes / (sum(ms) / 1e3) / 1e9
+
+    # ---- dominant kernel: rswa_decode_step (split-K + combine), eager launches
+    launch_ms, t_at = timed_decode_launches(rig, max(24, 2 * w.layers), flush)
+    per_launch_bytes = kv_bytes_per_layer(w, t_at)
+    dur = statistics.mean(launch_ms) / 1e3
+    achieved = per_launch_bytes / dur / 1e9
+
+    # ---- e2e through the public API with host buffers
+    e2e_ms, h2d, d2h = e2e_tokens(rig, args.steps, args.warmup, flush)
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([e2e_total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_total = float(tt.item())
+    e2e_value = world * args.steps / (e2e_total / 1e3)
+    pf_flops = prefill_flops_per_layer(w)
+    pf_mean = statistics.mean(pf_ms) / 1e3
+    assert rig.st.check() == 0, "device error word set during the run"
+    rig.st.close()
+    del rig
+    torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded N(0,1) q/k/v; random histories with a planted repeat)",
+        "config": {"workload": w.name, "batch": w.batch, "layers": w.layers, "heads": w.heads,
+                   "head_dim": w.head_dim, "prefill_len": list(w.prefill_lens)[:4],
+                   "window": w.window, "decode_steps_timed": args.steps,
+                   "decode_from_t": 0, "step": "one token: all layers' rswa_decode_step + "
+                   "rswa_advance + rswa_ngram_mask (n=35, window=128) as one CUDA graph",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world}"},
+        "kv_read_gbs": kv_gbs,
+        "roofline": {"kernel": "rswa_decode_step (decode_split_kernel + decode_combine_kernel)",
+                     "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_source": peak_src,
+                     "frac_of_datasheet_8000": achieved / DATASHEET_HBM_GBS,
+                     "algorithmic_bytes_per_launch": per_launch_bytes,
+                     "avg_launch_us": dur * 1e6, "traffic": None},
+        "prefill": {"workload": w.name, "tflops": pf_flops / pf_mean / 1e12, "unit": "TFLOP/s",
+                    "peak": tc_peak, "frac": pf_flops / pf_mean / 1e12 / tc_peak,
+                    "frac_of_datasheet_2250": pf_flops / pf_mean / 1e12 / DATASHEET_BF16_TFLOPS,
+                    "ms_per_layer": pf_mean * 1e3, "flops_per_layer": pf_flops},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (2 * w.layers + 2),
+        "clocks": clocks,
+    }
+
+    # ---- the bandwidth-bound workloads, steady state (t >= W), decode only
+    also = []
+    if world == 1 and args.also != "none":
+        for name in args.also.split(","):
+            also.append(run_also(synth.workload(name), args, flush, s, hbm_peak, tc_peak))
+            torch.cuda.empty_cache()
+        line["also"] = also
+
+    # ---- CPU oracle on this host (rank 0, N = 1)
+    if world == 1 and rank == 0 and args.cpu_seconds > 0:
+        rate, n, el, cores, lps = cpu_oracle_rate(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{n} decode steps x {lps} layers of {w.name} from t=0 "
+                                          f"(plus the n-gram ban) in {el:.1f} s"}
+    return line
+
+
+def run_also(w, args, flush, s, hbm_peak, tc_peak):
+    steps = args.also_steps
+    rig = DecodeRig(w, w.window, "random", s)
+    rig.capture()
+    ms, ts, _ = timed_tokens(rig, steps, args.warmup, flush)
+    kv_bytes = sum(w.layers * kv_bytes_per_layer(w, t) for t in ts)
+    launch_ms, t_at = timed_decode_launches(rig, 2 * w.layers, flush)
+    per_launch = kv_bytes_per_layer(w, t_at)
+    ach = per_launch / (statistics.mean(launch_ms) / 1e3) / 1e9
+    res = {"workload": w.name, "decode_steps_per_s": steps / (sum(ms) / 1e3),
+           "ms_per_step": sum(ms) / steps, "kv_read_gbs": kv_bytes / (sum(ms) / 1e3) / 1e9,
+           "decode_step_launch_gbs": ach, "frac_of_measured_hbm": ach / hbm_peak,
+           "frac_of_datasheet_8000": ach / DATASHEET_HBM_GBS, "avg_launch_us": statistics.mean(launch_ms) * 1e3,
+           "steps_timed": steps, "from_t": w.window if w.n_generated is None else "n_generated"}
+    assert rig.st.check() == 0
+    rig.st.close()
+    del rig
+    torch.cuda.empty_cache()
+    if w.name == "multi_page_decode" and not args.skip_prefill_also:
+        w1 = synth.Workload(w.name, w.cfg_id, w.dtype, w.batch, 2, w.heads, w.head_dim, w.window,
+                            w.prefill_lens, 0)
+        rig = DecodeRig(w1, 0, "prefill", s)
+        pf_ms = rig.prefill_all(flush)
+        f = prefill_flops_per_layer(w1) / (statistics.mean(pf_ms) / 1e3) / 1e12
+        res["prefill_tflops"] = f
+        res["prefill_frac"] = f / tc_peak
+        res["prefill_frac_of_datasheet_2250"] = f / DATASHEET_BF16_TFLOPS
+        rig.st.close()
+        del rig
+    return res
+
+
+def run_reference(args):
+    w = synth.workload(args.workload)
+    # size the sample: measure one step, then choose layers per step so that
+    # warmup + steps fit in the time budget
+    rate1, _, el1, _, _ = cpu_oracle_rate(w, 0.0, max_steps=1, layers_per_step=1)
+    per_layer = el1
+    budget = args.reference_budget
+    total_steps = args.steps + args.warmup
+    lps = max(1, min(w.layers, int(budget / max(per_layer * total_steps, 1e-9))))
+    if args.warmup:
+        cpu_oracle_rate(w, 0.0, max_steps=args.warmup, layers_per_step=lps)
+    rate, n, el, cores, lps = cpu_oracle_rate(w, 0.0, max_steps=args.steps, layers_per_step=lps)
+    return {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / n * 1e3 * (w.layers / lps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "batch": w.batch, "layers": w.layers,
+                                        "heads": w.heads, "head_dim": w.head_dim,
+                                        "prefill_len": list(w.prefill_lens)[:4], "window": w.window},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {lps} of {w.layers} layers of {w.name} "
+                                   f"(batch {w.batch}) + the n-gram ban; rate scaled to all layers"},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4096)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="single_page_decode")
+    ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving")
+    ap.add_argument("--also-steps", type=int, default=40)
+    ap.add_argument("--skip-prefill-also", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-budget", type=float, default=120.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        dist.barrier()
+    line = run_ours(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,209 @@
+/*
+ * librswa -- Reference Sliding Window Attention (R-SWA) decode hot path for
+ * NVIDIA B200 (sm_100a), behind a plain C ABI.
+ *
+ * Method source (cited by page title and section):
+ *   "开源5天Star破万之后：百度Unlimited-OCR的爆火路径复盘" (gtnt.cn)
+ *     §2.1 环形滑窗注意力 -- the KV cache keeps every prefill token at full
+ *          attention plus a ring of the W most recently generated tokens.
+ *          Generated tokens are appended until the cache holds prefill_len + W
+ *          entries; from then on each new token overwrites slot
+ *          prefill_len + ring_pos and ring_pos advances by one modulo W.  The
+ *          token then attends to the whole cache, whose size stays at
+ *          prefill_len + W however long the output runs.  W is
+ *          sliding_window_size = 128 in the model's config.
+ *     §2.3 反循环采样 -- inside a sliding window of the generated history,
+ *          every token that would repeat an n-gram of size ngram_size gets
+ *          score -inf (defaults no_repeat_ngram_size 35, ngram_window 128).
+ *     §三  -- the transformers path materialises the full prefill score
+ *          matrix; a flash-style ring implementation is named as open work.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named "device" are CUDA device pointers on the current device;
+ *    pointers named "host" are ordinary host memory.  `stream` is a
+ *    cudaStream_t (NULL = legacy default stream).  All device work is enqueued
+ *    asynchronously on `stream`; only rswa_state_create, rswa_get_ring and
+ *    rswa_check_device_error synchronise.
+ *  - OWNERSHIP: the caller owns ALL device memory (inputs, outputs, K/V
+ *    caches, workspace).  The library never allocates or frees device memory;
+ *    it keeps raw pointers inside the opaque host-side state.
+ *  - ERRORS: argument problems found on the host return RSWA_EINVAL before
+ *    anything is enqueued.  A failed launch returns RSWA_ECUDA.  Problems the
+ *    kernels find (a token id outside the vocabulary, a wait that ran out)
+ *    are recorded in a device error word and reported by
+ *    rswa_check_device_error (or, for rswa_ngram_mask, in the caller's
+ *    `device_error` word).  Nothing traps, aborts or waits without a bound.
+ *  - Element types: RSWA_BF16 (bfloat16, round-to-nearest-even outputs with
+ *    fp32 accumulation) or RSWA_F32.  head_dim is 64 or 128.
+ *  - Heads: multi-head attention, num_kv_heads == num_heads.  Positions (RoPE)
+ *    are the caller's business: keys are stored and used exactly as given.
+ *
+ * Layouts
+ * -------
+ *  Token-major activations: q, k, v, out of the prefill are packed varlen
+ *  [sum_b P_b][H][d]; decode q, k_new, v_new, out are [B][H][d]; rows are
+ *  contiguous, d fastest.
+ *
+ *  K/V cache of one layer (one buffer for K, one for V, rswa_cache_bytes()
+ *  each): sequence-major, then head-major, then slot:
+ *      element offset of (b, h, slot, e) =
+ *          (H * S_b + h * (P_b + W) + slot) * d + e,
+ *      S_b = sum_{b' < b} (P_b' + W),   0 <= slot < P_b + W.
+ *  Slots [0, P_b) hold the prefill; slots [P_b, P_b + W) hold the ring.
+ *  rswa_cache_offset() returns this offset.  Every (b, h) ring of the cache
+ *  is contiguous, so it is streamed with 16-byte-aligned bulk copies.
+ */
+#ifndef RSWA_H
+#define RSWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RSWA_ABI_VERSION 1
+
+typedef enum rswa_status {
+  RSWA_OK = 0,
+  RSWA_EINVAL = 1,   /* bad argument (null pointer, size, dtype, range)      */
+  RSWA_ENOMEM = 2,   /* caller-provided workspace smaller than required      */
+  RSWA_ECUDA = 3,    /* a CUDA runtime call or kernel launch failed          */
+  RSWA_ESTATE = 4,   /* call out of order (decode before prefill, ...)       */
+  RSWA_ETIMEOUT = 5, /* a kernel's bounded wait ran out (device error word)  */
+  RSWA_EDEVICE = 6   /* a kernel rejected its data (device error word)       */
+} rswa_status;
+
+typedef enum rswa_dtype { RSWA_F32 = 0, RSWA_BF16 = 1 } rswa_dtype;
+
+/* Model/batch shape shared by every layer. */
+typedef struct rswa_config {
+  int32_t batch;      /* B >= 1 sequences                                    */
+  int32_t num_layers; /* >= 1; each layer has its own K and V cache buffer   */
+  int32_t num_heads;  /* H >= 1                                              */
+  int32_t head_dim;   /* d in {64, 128}                                      */
+  int32_t window;     /* W >= 1 ring entries (the pages use 128)             */
+  int32_t dtype;      /* rswa_dtype of q/k/v/out and of the caches           */
+  float scale;        /* softmax scale; 0 selects 1/sqrt(head_dim)           */
+} rswa_config;
+
+/* Opaque host-side state: shape, raw device pointers, work decomposition. */
+typedef struct rswa_state rswa_state;
+
+/* Bytes of ONE cache buffer (K or V) of ONE layer:
+ *   H * d * elem_size * sum_b (P_b + W).
+ * prefill_len: host [B], each >= 0.  Returns 0 if the arguments are invalid. */
+size_t rswa_cache_bytes(const rswa_config *cfg, const int64_t *prefill_len);
+
+/* Bytes of device workspace rswa_state_create needs (error word, per-sequence
+ * counters, the split-K work list, split-K partials).  Depends on the device's
+ * SM count, so call it with the target device current.  0 if invalid. */
+size_t rswa_workspace_bytes(const rswa_config *cfg, const int64_t *prefill_len);
+
+/* Build the state for one batch.
+ *  prefill_len : host [B], P_b >= 0, P_b + W < 2^31.
+ *  n_generated : host [B] or NULL.  NULL: a fresh batch; every layer must be
+ *                filled by rswa_prefill before its first rswa_decode_step.
+ *                Non-NULL: resume a batch whose caches the caller has already
+ *                filled (prefill slots and the first min(n, W) ring slots, in
+ *                the layout above) after n_generated[b] tokens; decode may
+ *                start at once on every layer.
+ *  k_cache, v_cache : host arrays of num_layers device pointers, each to
+ *                rswa_cache_bytes() bytes, 16-byte aligned.
+ *  workspace   : device pointer to workspace_size >= rswa_workspace_bytes()
+ *                bytes, 256-byte aligned; owned by the caller, used by the
+ *                state until rswa_state_destroy.
+ *  stream      : the tables are uploaded on it; the call synchronises it.
+ *  out         : receives the new state.
+ * Returns RSWA_EINVAL, RSWA_ENOMEM (workspace too small) or RSWA_ECUDA. */
+rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len,
+                              const int64_t *n_generated, void *const *k_cache,
+                              void *const *v_cache, void *workspace, size_t workspace_size,
+                              void *stream, rswa_state **out);
+
+/* Free the host-side state.  Device memory stays the caller's. */
+rswa_status rswa_state_destroy(rswa_state *state);
+
+/* Element offset of (b, h, slot, 0) inside one layer's cache buffer, or -1. */
+int64_t rswa_cache_offset(const rswa_state *state, int32_t b, int32_t h, int64_t slot);
+
+/* Prefill of one layer [§2.1: the prefill segment keeps full attention].
+ *  q, k, v : device [sum_b P_b][H][d] (packed varlen, sequence b's tokens at
+ *            rows sum_{b'<b} P_b' ...), dtype of the config.
+ *  out     : device [sum_b P_b][H][d]: causal softmax attention of each token
+ *            over tokens 0..i of its own sequence (no window).
+ * Also stores k, v into cache slots [0, P_b) of this layer; the ring
+ * counters are not touched.  All pointers 16-byte aligned.  Returns
+ * RSWA_EINVAL for a bad layer or pointer. */
+rswa_status rswa_prefill(rswa_state *state, int32_t layer, const void *q, const void *k,
+                         const void *v, void *out, void *stream);
+
+/* One decode step of one layer [§2.1 steady-state/warm-up phases].
+ *  q, k_new, v_new, out : device [B][H][d].
+ * For each sequence b with t_b tokens generated so far (t_b is device
+ * resident, advanced by rswa_advance):
+ *   slot  = P_b + (t_b mod W)     -- the warm-up append and the steady-state
+ *                                    ring overwrite are the same formula;
+ *   cache[slot] <- (k_new, v_new);
+ *   out   = softmax attention of q over slots [0, P_b + min(t_b + 1, W)).
+ * The write and the attention are one fused split-K kernel followed by a
+ * combine kernel.  Safe to capture in a CUDA graph (no host-side state
+ * changes per step).  RSWA_ESTATE if the layer was never prefilled. */
+rswa_status rswa_decode_step(rswa_state *state, int32_t layer, const void *q, const void *k_new,
+                             const void *v_new, void *out, void *stream);
+
+/* t_b += 1 for every sequence, on the device: once per generated token, after
+ * the token's last layer.  Capturable in a CUDA graph. */
+rswa_status rswa_advance(rswa_state *state, void *stream);
+
+/* Restore every t_b to its value at rswa_state_create (0, or n_generated),
+ * on the device; capturable.  Starts the batch's generation over without
+ * rebuilding the state (the caches are not touched). */
+rswa_status rswa_reset_ring(rswa_state *state, void *stream);
+
+/* Windowed no-repeat n-gram ban [§2.3].
+ *  logits     : device fp32 [rows][ld], ld >= vocab; modified in place.
+ *  history    : device int32 [rows][hist_ld], hist_ld >= window; row r holds
+ *               its last h_r generated tokens, oldest first, in [0, h_r).
+ *  hist_len   : device int32 [rows] (h_r, 0 <= h_r <= window) or NULL (all
+ *               rows hold `window` tokens).
+ *  n          : n-gram size >= 1 (the pages use 35); window >= 0 (128).
+ *  device_error : device int32 or NULL; on bad row data the kernel ORs
+ *               RSWA_DEVERR_BAD_TOKEN / RSWA_DEVERR_BAD_LENGTH into it.
+ * For each row with h_r >= n: the next token x would form the n-gram
+ * (hist[h_r-n+1 .. h_r-1], x); every start i in [0, h_r - n] whose (n-1)-gram
+ * hist[i .. i+n-2] equals that prefix sets logits[r][hist[i+n-1]] = -inf.
+ * Nothing else is written, bit for bit.  A row with h_r outside [0, window]
+ * or a token outside [0, vocab) in [0, h_r) is left untouched.  Rows with
+ * h_r < n, and window < n, ban nothing. */
+rswa_status rswa_ngram_mask(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                            const int32_t *hist_len, int32_t rows, int32_t vocab, int32_t n,
+                            int32_t window, int32_t *device_error, void *stream);
+
+/* Synchronises `stream`, then copies the ring counters to the host:
+ *  n_generated : host [B] or NULL -- t_b;
+ *  ring_pos    : host [B] or NULL -- the pages' ring_pos: 0 during warm-up,
+ *                t_b mod W once the cache is full (next slot is P_b+ring_pos);
+ *  cache_len   : host [B] or NULL -- entries held, P_b + min(t_b, W). */
+rswa_status rswa_get_ring(const rswa_state *state, int64_t *n_generated, int32_t *ring_pos,
+                          int64_t *cache_len, void *stream);
+
+/* Synchronises `stream` and reads the state's device error word:
+ * RSWA_OK, RSWA_ETIMEOUT or RSWA_EDEVICE.  Clears the word. */
+rswa_status rswa_check_device_error(rswa_state *state, void *stream);
+
+/* Static description of a status code. */
+const char *rswa_status_string(rswa_status status);
+
+/* Bits of a device error word. */
+#define RSWA_DEVERR_TIMEOUT 1
+#define RSWA_DEVERR_BAD_TOKEN 2
+#define RSWA_DEVERR_BAD_LENGTH 4
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSWA_H */

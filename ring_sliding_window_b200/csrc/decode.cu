@@ -1,0 +1,377 @@
+// R-SWA decode step: fused ring-slot write + split-K attention over the
+// whole cache, then a log-sum-exp combine of the split partials.
+//
+// Method ("开源5天Star破万之后：百度Unlimited-OCR的爆火路径复盘", §2.1): each
+// generated token's K/V goes to slot prefill_len + ring_pos (an append during
+// warm-up, an overwrite once the cache holds prefill_len + W entries), and the
+// token then attends to every entry of the cache.
+//
+// Design (HBM-bound: every cached K/V byte is read once per step):
+//  - Work is split "stream-K" style: the flattened key rows of all (b, h)
+//    rings are cut into equal contiguous ranges, one per CTA, so every CTA
+//    streams the same number of bytes whatever the batch's raggedness.  A
+//    CTA's range is a list of pieces, one per (b, h) ring it touches.
+//  - One producer lane streams K and V rows into a 4-stage shared-memory ring
+//    with bulk copies (cp.async.bulk, the TMA engine) completing on mbarriers;
+//    four consumer warps compute.  The producer runs ahead across piece
+//    boundaries so the copy pipeline never drains inside a CTA.
+//  - Each row is handled by 8 lanes (16-byte chunks interleaved so a quarter
+//    warp reads 128 contiguous bytes: no bank conflicts); the dot product is a
+//    3-step xor-shuffle; softmax runs online in the log2 domain (exp2f).
+//  - The CTA whose piece holds this step's write slot stores k_new/v_new to
+//    the cache and substitutes them for that row from shared memory, so no CTA
+//    ever uses the stale slot and nobody re-reads the fresh one.
+//  - Each piece ends in an unnormalised partial (m, l, o[d]); the combine
+//    kernel merges the pieces of each (b, h).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace rswa {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T, int D>
+struct DecodeShape {
+  static constexpr int kRowBytes = D * (int)sizeof(T);
+  static constexpr int kStageRows = 8192 / kRowBytes;  // 8 KB of K (and of V) per stage
+  static constexpr int kStages = 4;
+  static constexpr int kConsumerWarps = 4;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int kGroups = kConsumerWarps * 4;  // 8 lanes per row
+  static constexpr int kPasses = kStageRows / kGroups;
+  static constexpr int kChunks = kRowBytes / 16;
+  static constexpr int kChunksPerLane = kChunks / 8;
+  static constexpr int kElemPerChunk = 16 / (int)sizeof(T);
+  static constexpr int kEPL = kChunksPerLane * kElemPerChunk;  // elements per lane
+  static_assert(kStageRows % kGroups == 0, "stage rows must split over the groups");
+  static_assert(kChunks % 8 == 0, "row must be a multiple of 8 chunks");
+  static_assert(kEPL * 8 == D, "lane split must cover the row");
+};
+
+template <typename T, int D>
+struct __align__(128) DecodeSmem {
+  using S = DecodeShape<T, D>;
+  uint8_t k[S::kStages][S::kStageRows * S::kRowBytes];
+  uint8_t v[S::kStages][S::kStageRows * S::kRowBytes];
+  uint8_t sub_k[S::kRowBytes];
+  uint8_t sub_v[S::kRowBytes];
+  float red_o[S::kGroups][D];
+  float red_m[S::kGroups];
+  float red_l[S::kGroups];
+  uint64_t full[S::kStages];
+  uint64_t empty[S::kStages];
+};
+
+struct DecodeArgs {
+  DeviceView v;
+  const void *q, *k_new, *v_new;
+  void *kc, *vc;
+};
+
+__device__ __forceinline__ int64_t seg_offset_rows(const DeviceView &v, int b, int h, int plen) {
+  // first row (slot 0) of ring (b, h) in units of rows
+  return (int64_t)v.H * v.slot_base[b] + (int64_t)h * (plen + v.W);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
+    decode_split_kernel(const DecodeArgs a) {
+  using S = DecodeShape<T, D>;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  DecodeSmem<T, D> &sm = *reinterpret_cast<DecodeSmem<T, D> *>(smem_raw);
+  const DeviceView &v = a.v;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int p_begin = v.cta_piece[blockIdx.x];
+  const int p_end = v.cta_piece[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], S::kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == S::kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    int stage = 0;
+    uint32_t round = 0;
+    bool dead = false;
+    for (int p = p_begin; p < p_end && !dead; ++p) {
+      const DecodePiece pc = v.pieces[p];
+      const int b = pc.bh / v.H, h = pc.bh % v.H;
+      const int plen = v.plen[b];
+      const int64_t t = v.t[b];
+      const int valid = plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
+      const int ke = pc.key_end < valid ? pc.key_end : valid;
+      const int64_t row0 = seg_offset_rows(v, b, h, plen);
+      const uint8_t *kbase = (const uint8_t *)a.kc + row0 * S::kRowBytes;
+      const uint8_t *vbase = (const uint8_t *)a.vc + row0 * S::kRowBytes;
+      for (int k0 = pc.key_begin; k0 < ke; k0 += S::kStageRows) {
+        const int rows = (ke - k0) < S::kStageRows ? (ke - k0) : S::kStageRows;
+        if (!mbar_wait_bounded(&sm.empty[stage], (round & 1) ^ 1, v.err, RSWA_DEVERR_TIMEOUT)) {
+          dead = true;
+          break;
+        }
+        const uint32_t bytes = (uint32_t)rows * S::kRowBytes;
+        mbar_arrive_expect_tx(&sm.full[stage], 2 * bytes);
+        bulk_g2s(sm.k[stage], kbase + (int64_t)k0 * S::kRowBytes, bytes, &sm.full[stage]);
+        bulk_g2s(sm.v[stage], vbase + (int64_t)k0 * S::kRowBytes, bytes, &sm.full[stage]);
+        if (++stage == S::kStages) {
+          stage = 0;
+          ++round;
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int tid = threadIdx.x;  // 0..127
+  const int g = warp * 4 + (lane >> 3);
+  const int li = lane & 7;
+  int stage = 0;
+  uint32_t round = 0;
+  bool dead = false;
+
+  for (int p = p_begin; p < p_end; ++p) {
+    const DecodePiece pc = v.pieces[p];
+    const int b = pc.bh / v.H, h = pc.bh % v.H;
+    const int plen = v.plen[b];
+    const int64_t t = v.t[b];
+    const int valid = plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
+    const int wslot = plen + (int)(t % v.W);
+    const int ke = pc.key_end < valid ? pc.key_end : valid;
+    const bool owner = wslot >= pc.key_begin && wslot < pc.key_end;
+    const int64_t in_off = ((int64_t)b * v.H + h) * D;  // element offset into [B][H][D]
+
+    // q slice of this lane, pre-scaled into the log2 domain
+    float qf[S::kEPL];
+    {
+      const uint8_t *qrow = (const uint8_t *)a.q + in_off * (int64_t)sizeof(T);
+#pragma unroll
+      for (int j = 0; j < S::kChunksPerLane; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(qrow + (li + 8 * j) * 16);
+        Chunk<T>::widen(u, qf + j * S::kElemPerChunk);
+      }
+      const float qs = v.scale * kLog2e;
+#pragma unroll
+      for (int e = 0; e < S::kEPL; ++e) qf[e] *= qs;
+    }
+
+    if (owner) {
+      // ring write of this step + shared-memory copy for the substitution
+      const uint8_t *kn = (const uint8_t *)a.k_new + in_off * (int64_t)sizeof(T);
+      const uint8_t *vn = (const uint8_t *)a.v_new + in_off * (int64_t)sizeof(T);
+      const int64_t wrow = seg_offset_rows(v, b, h, plen) + wslot;
+      uint8_t *kdst = (uint8_t *)a.kc + wrow * S::kRowBytes;
+      uint8_t *vdst = (uint8_t *)a.vc + wrow * S::kRowBytes;
+      for (int c = tid; c < 2 * S::kChunks; c += 128) {
+        const bool isk = c < S::kChunks;
+        const int cc = isk ? c : c - S::kChunks;
+        const uint4 u = *reinterpret_cast<const uint4 *>((isk ? kn : vn) + cc * 16);
+        *reinterpret_cast<uint4 *>((isk ? sm.sub_k : sm.sub_v) + cc * 16) = u;
+        *reinterpret_cast<uint4 *>((isk ? kdst : vdst) + cc * 16) = u;
+      }
+      named_bar_sync(1, 128);
+    }
+
+    float m = -INFINITY, l = 0.f;
+    float o[S::kEPL];
+#pragma unroll
+    for (int e = 0; e < S::kEPL; ++e) o[e] = 0.f;
+
+    for (int k0 = pc.key_begin; k0 < ke; k0 += S::kStageRows) {
+      const int rows = (ke - k0) < S::kStageRows ? (ke - k0) : S::kStageRows;
+      if (!dead && !mbar_wait_bounded(&sm.full[stage], round & 1, v.err, RSWA_DEVERR_TIMEOUT))
+        dead = true;
+      if (!dead) {
+        const uint8_t *ks = sm.k[stage];
+        const uint8_t *vs = sm.v[stage];
+        float sc[S::kPasses];
+#pragma unroll
+        for (int ps = 0; ps < S::kPasses; ++ps) {
+          const int r = ps * S::kGroups + g;
+          float acc = 0.f;
+          if (r < rows) {
+            const uint8_t *krow = (owner && k0 + r == wslot) ? sm.sub_k : ks + r * S::kRowBytes;
+#pragma unroll
+            for (int j = 0; j < S::kChunksPerLane; ++j) {
+              const uint4 u = *reinterpret_cast<const uint4 *>(krow + (li + 8 * j) * 16);
+              float kf[S::kElemPerChunk];
+              Chunk<T>::widen(u, kf);
+#pragma unroll
+              for (int e = 0; e < S::kElemPerChunk; ++e)
+                acc = fmaf(qf[j * S::kElemPerChunk + e], kf[e], acc);
+            }
+          }
+          acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+          sc[ps] = r < rows ? acc : -INFINITY;
+        }
+        float m_new = m;
+#pragma unroll
+        for (int ps = 0; ps < S::kPasses; ++ps) m_new = fmaxf(m_new, sc[ps]);
+        if (m_new != -INFINITY) {
+          const float corr = exp2f(m - m_new);
+          l *= corr;
+#pragma unroll
+          for (int e = 0; e < S::kEPL; ++e) o[e] *= corr;
+#pragma unroll
+          for (int ps = 0; ps < S::kPasses; ++ps) {
+            const int r = ps * S::kGroups + g;
+            if (r < rows) {
+              const float pr = exp2f(sc[ps] - m_new);
+              l += pr;
+              const uint8_t *vrow = (owner && k0 + r == wslot) ? sm.sub_v : vs + r * S::kRowBytes;
+#pragma unroll
+              for (int j = 0; j < S::kChunksPerLane; ++j) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(vrow + (li + 8 * j) * 16);
+                float vf[S::kElemPerChunk];
+                Chunk<T>::widen(u, vf);
+#pragma unroll
+                for (int e = 0; e < S::kElemPerChunk; ++e)
+                  o[j * S::kElemPerChunk + e] = fmaf(pr, vf[e], o[j * S::kElemPerChunk + e]);
+              }
+            }
+          }
+          m = m_new;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[stage]);
+      if (++stage == S::kStages) {
+        stage = 0;
+        ++round;
+      }
+    }
+
+    // -------- piece end: merge the 16 group states into one partial
+    if (li == 0) {
+      sm.red_m[g] = m;
+      sm.red_l[g] = l;
+    }
+#pragma unroll
+    for (int j = 0; j < S::kChunksPerLane; ++j)
+#pragma unroll
+      for (int e = 0; e < S::kElemPerChunk; ++e)
+        sm.red_o[g][(li + 8 * j) * S::kElemPerChunk + e] = o[j * S::kElemPerChunk + e];
+    named_bar_sync(1, 128);
+    float M = -INFINITY;
+#pragma unroll
+    for (int gg = 0; gg < S::kGroups; ++gg) M = fmaxf(M, sm.red_m[gg]);
+    for (int e = tid; e < D; e += 128) {
+      float acc = 0.f;
+      if (M != -INFINITY)
+#pragma unroll
+        for (int gg = 0; gg < S::kGroups; ++gg)
+          acc = fmaf(sm.red_o[gg][e], exp2f(sm.red_m[gg] - M), acc);
+      v.part_o[(int64_t)p * D + e] = acc;
+    }
+    if (tid == 0) {
+      float L = 0.f;
+      if (M != -INFINITY)
+        for (int gg = 0; gg < S::kGroups; ++gg) L = fmaf(sm.red_l[gg], exp2f(sm.red_m[gg] - M), L);
+      v.part_ml[p] = make_float2(M, L);
+    }
+    named_bar_sync(1, 128);
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const DeviceView v, T *out) {
+  const int bh = blockIdx.x;
+  const int e = threadIdx.x;
+  const int p0 = v.bh_piece[bh], p1 = v.bh_piece[bh + 1];
+  float M = -INFINITY;
+  for (int p = p0; p < p1; ++p) {
+    const float2 ml = v.part_ml[p];
+    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  }
+  float L = 0.f, acc = 0.f;
+  for (int p = p0; p < p1; ++p) {
+    const float2 ml = v.part_ml[p];
+    if (ml.y > 0.f) {
+      const float w = exp2f(ml.x - M);
+      L = fmaf(w, ml.y, L);
+      acc = fmaf(w, v.part_o[(int64_t)p * D + e], acc);
+    }
+  }
+  out[(int64_t)bh * D + e] = from_float<T>(acc / L);
+}
+
+__global__ void advance_kernel(int64_t *t, int B) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) t[b] += 1;
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_t(const DeviceView &v, const void *q, const void *k_new,
+                            const void *v_new, void *kc, void *vc, void *out, cudaStream_t s) {
+  using S = DecodeShape<T, D>;
+  const int smem = (int)sizeof(DecodeSmem<T, D>);
+  static bool attr_set = false;  // per (T, D) instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  DecodeArgs a{v, q, k_new, v_new, kc, vc};
+  decode_split_kernel<T, D><<<v.decode_grid, S::kThreads, smem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<T, D><<<v.B * v.H, D, 0, s>>>(v, (T *)out);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+int ctas_per_sm_t() {
+  using S = DecodeShape<T, D>;
+  const int smem = (int)sizeof(DecodeSmem<T, D>);
+  if (cudaFuncSetAttribute(decode_split_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<T, D>, S::kThreads,
+                                                    smem) != cudaSuccess ||
+      n < 1)
+    return 1;
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
+                          const void *v_new, void *kc, void *vc, void *out, cudaStream_t s) {
+  if (v.dtype == RSWA_BF16) {
+    if (v.D == 128)
+      return launch_decode_t<__nv_bfloat16, 128>(v, q, k_new, v_new, kc, vc, out, s);
+    return launch_decode_t<__nv_bfloat16, 64>(v, q, k_new, v_new, kc, vc, out, s);
+  }
+  if (v.D == 128) return launch_decode_t<float, 128>(v, q, k_new, v_new, kc, vc, out, s);
+  return launch_decode_t<float, 64>(v, q, k_new, v_new, kc, vc, out, s);
+}
+
+cudaError_t launch_advance(const DeviceView &v, cudaStream_t s) {
+  advance_kernel<<<(v.B + 255) / 256, 256, 0, s>>>(v.t, v.B);
+  return cudaGetLastError();
+}
+
+int decode_ctas_per_sm(int dtype, int head_dim) {
+  if (dtype == RSWA_BF16)
+    return head_dim == 128 ? ctas_per_sm_t<__nv_bfloat16, 128>() : ctas_per_sm_t<__nv_bfloat16, 64>();
+  return head_dim == 128 ? ctas_per_sm_t<float, 128>() : ctas_per_sm_t<float, 64>();
+}
+
+}  // namespace rswa

@@ -1,0 +1,113 @@
+// Internal declarations shared by the librswa host layer and its kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/rswa.h"
+
+namespace rswa {
+
+// Split-K piece of the decode attention: keys [key_begin, key_end) of one
+// (b, h) ring, all processed by one CTA.  Pieces are listed in flattened
+// (b, h, key) order, so the pieces of one (b, h) are contiguous.
+struct DecodePiece {
+  int32_t bh;
+  int32_t key_begin;
+  int32_t key_end;
+  int32_t cta;
+};
+
+// Byte offsets of the workspace sections (each 256-byte aligned).
+struct WsLayout {
+  size_t err;        // int32 device error word (+ int32 debug flags)
+  size_t t;          // int64 [B]   tokens generated so far
+  size_t plen;       // int32 [B]   P_b
+  size_t slot_base;  // int64 [B+1] sum_{b'<b} (P_b' + W)
+  size_t tok_base;   // int64 [B+1] sum_{b'<b} P_b'
+  size_t tile_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kPrefillTile)
+  size_t tile64_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kSimtTile)
+  size_t pieces;     // DecodePiece [n_pieces]
+  size_t cta_piece;  // int32 [G+1] first piece of each decode CTA
+  size_t bh_piece;   // int32 [B*H+1] first piece of each (b, h)
+  size_t part_ml;    // float2 [n_pieces] (running max in log2 units, sum)
+  size_t part_o;     // float [n_pieces][d] unnormalised outputs
+  size_t total;
+};
+
+// Host-side plan of the decode decomposition (depends on the SM count).
+struct DecodePlan {
+  int grid;      // decode CTAs
+  int n_pieces;  // total pieces
+  std::vector<DecodePiece> pieces;
+  std::vector<int32_t> cta_piece;  // [grid + 1]
+  std::vector<int32_t> bh_piece;   // [B*H + 1]
+};
+
+constexpr int kPrefillTile = 128;  // query rows per prefill tile (tensor-core kernel)
+constexpr int kSimtTile = 64;      // query rows per prefill tile (FP32 SIMT kernel)
+
+// Everything the kernels need, as plain device pointers.
+struct DeviceView {
+  int B, H, D, W, L;
+  int dtype;
+  float scale;
+  int *err;
+  int64_t *t;
+  const int32_t *plen;
+  const int64_t *slot_base;
+  const int64_t *tok_base;
+  const int32_t *tile_base;
+  const int32_t *tile64_base;
+  const DecodePiece *pieces;
+  const int32_t *cta_piece;
+  const int32_t *bh_piece;
+  float2 *part_ml;
+  float *part_o;
+  int decode_grid;
+  int n_pieces;
+  int64_t total_tokens;  // sum P_b
+  int total_tiles;       // sum ceil(P_b / kPrefillTile)
+  int total_tiles64;     // sum ceil(P_b / kSimtTile)
+  int max_plen;
+};
+
+}  // namespace rswa
+
+struct rswa_state {
+  rswa_config cfg;
+  std::vector<int64_t> plen;
+  std::vector<void *> k_cache, v_cache;
+  std::vector<uint8_t> layer_ready;  // prefilled or resumed
+  void *workspace;
+  size_t workspace_size;
+  int device;
+  int num_sms;
+  rswa::WsLayout ws;
+  rswa::DecodePlan plan;
+  rswa::DeviceView dv;
+};
+
+namespace rswa {
+
+// Launchers (return cudaGetLastError() of their launch).
+cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
+                          const void *v_new, void *kc, void *vc, void *out, cudaStream_t s);
+cudaError_t launch_advance(const DeviceView &v, cudaStream_t s);
+cudaError_t launch_cache_fill(const DeviceView &v, const void *k, const void *vv, void *kc,
+                              void *vc, cudaStream_t s);
+cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,
+                                const void *vv, void *out, cudaStream_t s);
+cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
+                              void *out, cudaStream_t s);
+cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                         const int32_t *hist_len, int rows, int vocab, int n, int window,
+                         int *err, cudaStream_t s);
+
+// Resident decode CTAs per SM for (dtype, head_dim); used by the planner.
+int decode_ctas_per_sm(int dtype, int head_dim);
+
+}  // namespace rswa

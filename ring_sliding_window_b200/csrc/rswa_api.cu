@@ -1,0 +1,358 @@
+// librswa host layer: argument checks, the split-K work plan, the workspace
+// layout, and the exported C entry points declared in include/rswa.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "internal.h"
+
+using namespace rswa;
+
+namespace {
+
+constexpr int64_t kMinRowsPerCta = 64;  // below this a decode CTA is mostly latency
+
+bool config_ok(const rswa_config *c, const int64_t *plen) {
+  if (!c || !plen) return false;
+  if (c->batch < 1 || c->num_layers < 1 || c->num_heads < 1 || c->window < 1) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->dtype != RSWA_F32 && c->dtype != RSWA_BF16) return false;
+  if (!(c->scale >= 0.f) || !isfinite(c->scale)) return false;
+  int64_t rows = 0;
+  for (int b = 0; b < c->batch; ++b) {
+    if (plen[b] < 0 || plen[b] + c->window >= (int64_t(1) << 31)) return false;
+    rows += (plen[b] + c->window) * c->num_heads;
+    if (rows >= (int64_t(1) << 40)) return false;
+  }
+  return true;
+}
+
+size_t elem_size(const rswa_config *c) { return c->dtype == RSWA_BF16 ? 2 : 4; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int current_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+int sm_count(int dev) {
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 148;
+  return n;
+}
+
+// Equal contiguous ranges of the flattened (b, h, key) rows, one per CTA.
+DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, int ctas_per_sm) {
+  const int B = c->batch, H = c->num_heads, W = c->window;
+  std::vector<int64_t> seg_start((size_t)B * H + 1, 0);
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h)
+      seg_start[(size_t)b * H + h + 1] = seg_start[(size_t)b * H + h] + plen[b] + W;
+  const int64_t R = seg_start.back();
+  int64_t G = std::min<int64_t>((int64_t)num_sms * ctas_per_sm, (R + kMinRowsPerCta - 1) / kMinRowsPerCta);
+  if (G < 1) G = 1;
+  const int64_t rpc = (R + G - 1) / G;
+  G = (R + rpc - 1) / rpc;
+
+  DecodePlan p;
+  p.grid = (int)G;
+  p.cta_piece.assign((size_t)G + 1, 0);
+  p.bh_piece.assign((size_t)B * H + 1, 0);
+  size_t seg = 0;
+  for (int64_t cta = 0; cta < G; ++cta) {
+    p.cta_piece[(size_t)cta] = (int32_t)p.pieces.size();
+    int64_t r0 = cta * rpc;
+    const int64_t r1 = std::min(R, r0 + rpc);
+    while (r0 < r1) {
+      while (seg_start[seg + 1] <= r0) ++seg;
+      const int64_t e = std::min(r1, seg_start[seg + 1]);
+      DecodePiece pc;
+      pc.bh = (int32_t)seg;
+      pc.key_begin = (int32_t)(r0 - seg_start[seg]);
+      pc.key_end = (int32_t)(e - seg_start[seg]);
+      pc.cta = (int32_t)cta;
+      p.pieces.push_back(pc);
+      r0 = e;
+    }
+  }
+  p.cta_piece[(size_t)G] = (int32_t)p.pieces.size();
+  p.n_pieces = (int)p.pieces.size();
+  // first piece of each (b, h): pieces are in flattened order
+  size_t i = 0;
+  for (size_t bh = 0; bh <= (size_t)B * H; ++bh) {
+    while (i < p.pieces.size() && (size_t)p.pieces[i].bh < bh) ++i;
+    p.bh_piece[bh] = (int32_t)i;
+  }
+  return p;
+}
+
+WsLayout layout_ws(const rswa_config *c, const DecodePlan &p) {
+  const size_t B = (size_t)c->batch;
+  WsLayout w;
+  size_t off = 0;
+  w.err = off;         off = align256(off + 2 * sizeof(int32_t));
+  w.t = off;           off = align256(off + 2 * B * sizeof(int64_t));  // t and its reset copy
+  w.plen = off;        off = align256(off + B * sizeof(int32_t));
+  w.slot_base = off;   off = align256(off + (B + 1) * sizeof(int64_t));
+  w.tok_base = off;    off = align256(off + (B + 1) * sizeof(int64_t));
+  w.tile_base = off;   off = align256(off + (B + 1) * sizeof(int32_t));
+  w.tile64_base = off; off = align256(off + (B + 1) * sizeof(int32_t));
+  w.pieces = off;      off = align256(off + (size_t)p.n_pieces * sizeof(DecodePiece));
+  w.cta_piece = off;   off = align256(off + ((size_t)p.grid + 1) * sizeof(int32_t));
+  w.bh_piece = off;    off = align256(off + (B * c->num_heads + 1) * sizeof(int32_t));
+  w.part_ml = off;     off = align256(off + (size_t)p.n_pieces * sizeof(float2));
+  w.part_o = off;      off = align256(off + (size_t)p.n_pieces * c->head_dim * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+rswa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RSWA_OK : RSWA_ECUDA; }
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+extern "C" {
+
+size_t rswa_cache_bytes(const rswa_config *cfg, const int64_t *prefill_len) {
+  if (!config_ok(cfg, prefill_len)) return 0;
+  size_t slots = 0;
+  for (int b = 0; b < cfg->batch; ++b) slots += (size_t)(prefill_len[b] + cfg->window);
+  return slots * (size_t)cfg->num_heads * (size_t)cfg->head_dim * elem_size(cfg);
+}
+
+size_t rswa_workspace_bytes(const rswa_config *cfg, const int64_t *prefill_len) {
+  if (!config_ok(cfg, prefill_len)) return 0;
+  const int dev = current_device();
+  if (dev < 0) return 0;
+  const DecodePlan p =
+      plan_decode(cfg, prefill_len, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+  return layout_ws(cfg, p).total;
+}
+
+rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len,
+                              const int64_t *n_generated, void *const *k_cache,
+                              void *const *v_cache, void *workspace, size_t workspace_size,
+                              void *stream, rswa_state **out) {
+  if (!out) return RSWA_EINVAL;
+  *out = nullptr;
+  if (!config_ok(cfg, prefill_len) || !k_cache || !v_cache || !workspace) return RSWA_EINVAL;
+  if (((uintptr_t)workspace & 255u) != 0) return RSWA_EINVAL;
+  for (int l = 0; l < cfg->num_layers; ++l)
+    if (!k_cache[l] || !v_cache[l] || !aligned16(k_cache[l]) || !aligned16(v_cache[l]))
+      return RSWA_EINVAL;
+  if (n_generated)
+    for (int b = 0; b < cfg->batch; ++b)
+      if (n_generated[b] < 0) return RSWA_EINVAL;
+  const int dev = current_device();
+  if (dev < 0) return RSWA_ECUDA;
+
+  rswa_state *s = new (std::nothrow) rswa_state();
+  if (!s) return RSWA_ENOMEM;
+  s->cfg = *cfg;
+  if (s->cfg.scale == 0.f) s->cfg.scale = 1.0f / sqrtf((float)cfg->head_dim);
+  s->plen.assign(prefill_len, prefill_len + cfg->batch);
+  s->k_cache.assign(k_cache, k_cache + cfg->num_layers);
+  s->v_cache.assign(v_cache, v_cache + cfg->num_layers);
+  s->layer_ready.assign((size_t)cfg->num_layers, n_generated ? 1 : 0);
+  s->workspace = workspace;
+  s->workspace_size = workspace_size;
+  s->device = dev;
+  s->num_sms = sm_count(dev);
+  s->plan = plan_decode(cfg, prefill_len, s->num_sms, decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+  s->ws = layout_ws(cfg, s->plan);
+  if (workspace_size < s->ws.total) {
+    delete s;
+    return RSWA_ENOMEM;
+  }
+
+  // host images of the tables
+  const int B = cfg->batch;
+  std::vector<uint8_t> img(s->ws.total, 0);
+  auto at = [&](size_t off) { return img.data() + off; };
+  int64_t *t = (int64_t *)at(s->ws.t);
+  int32_t *pl = (int32_t *)at(s->ws.plen);
+  int64_t *sb = (int64_t *)at(s->ws.slot_base);
+  int64_t *tb = (int64_t *)at(s->ws.tok_base);
+  int32_t *tl = (int32_t *)at(s->ws.tile_base);
+  int32_t *tl64 = (int32_t *)at(s->ws.tile64_base);
+  int max_plen = 0;
+  for (int b = 0; b < B; ++b) {
+    t[b] = n_generated ? n_generated[b] : 0;
+    t[B + b] = t[b];  // reset copy
+    pl[b] = (int32_t)prefill_len[b];
+    sb[b + 1] = sb[b] + prefill_len[b] + cfg->window;
+    tb[b + 1] = tb[b] + prefill_len[b];
+    tl[b + 1] = tl[b] + (int32_t)((prefill_len[b] + kPrefillTile - 1) / kPrefillTile);
+    tl64[b + 1] = tl64[b] + (int32_t)((prefill_len[b] + kSimtTile - 1) / kSimtTile);
+    max_plen = std::max(max_plen, (int)prefill_len[b]);
+  }
+  memcpy(at(s->ws.pieces), s->plan.pieces.data(), s->plan.pieces.size() * sizeof(DecodePiece));
+  memcpy(at(s->ws.cta_piece), s->plan.cta_piece.data(), s->plan.cta_piece.size() * sizeof(int32_t));
+  memcpy(at(s->ws.bh_piece), s->plan.bh_piece.data(), s->plan.bh_piece.size() * sizeof(int32_t));
+  // upload everything up to the partials (which the kernels overwrite)
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(workspace, img.data(), s->ws.part_ml, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    delete s;
+    return RSWA_ECUDA;
+  }
+
+  uint8_t *w = (uint8_t *)workspace;
+  DeviceView &v = s->dv;
+  v.B = B;
+  v.H = cfg->num_heads;
+  v.D = cfg->head_dim;
+  v.W = cfg->window;
+  v.L = cfg->num_layers;
+  v.dtype = cfg->dtype;
+  v.scale = s->cfg.scale;
+  v.err = (int *)(w + s->ws.err);
+  v.t = (int64_t *)(w + s->ws.t);
+  v.plen = (const int32_t *)(w + s->ws.plen);
+  v.slot_base = (const int64_t *)(w + s->ws.slot_base);
+  v.tok_base = (const int64_t *)(w + s->ws.tok_base);
+  v.tile_base = (const int32_t *)(w + s->ws.tile_base);
+  v.tile64_base = (const int32_t *)(w + s->ws.tile64_base);
+  v.pieces = (const DecodePiece *)(w + s->ws.pieces);
+  v.cta_piece = (const int32_t *)(w + s->ws.cta_piece);
+  v.bh_piece = (const int32_t *)(w + s->ws.bh_piece);
+  v.part_ml = (float2 *)(w + s->ws.part_ml);
+  v.part_o = (float *)(w + s->ws.part_o);
+  v.decode_grid = s->plan.grid;
+  v.n_pieces = s->plan.n_pieces;
+  v.total_tokens = tb[B];
+  v.total_tiles = tl[B];
+  v.total_tiles64 = tl64[B];
+  v.max_plen = max_plen;
+  *out = s;
+  return RSWA_OK;
+}
+
+rswa_status rswa_state_destroy(rswa_state *state) {
+  if (!state) return RSWA_EINVAL;
+  delete state;
+  return RSWA_OK;
+}
+
+int64_t rswa_cache_offset(const rswa_state *s, int32_t b, int32_t h, int64_t slot) {
+  if (!s || b < 0 || b >= s->cfg.batch || h < 0 || h >= s->cfg.num_heads) return -1;
+  const int64_t P = s->plen[(size_t)b];
+  if (slot < 0 || slot >= P + s->cfg.window) return -1;
+  int64_t base = 0;
+  for (int i = 0; i < b; ++i) base += s->plen[(size_t)i] + s->cfg.window;
+  return ((int64_t)s->cfg.num_heads * base + (int64_t)h * (P + s->cfg.window) + slot) *
+         s->cfg.head_dim;
+}
+
+rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void *k,
+                         const void *v, void *out, void *stream) {
+  if (!s || layer < 0 || layer >= s->cfg.num_layers) return RSWA_EINVAL;
+  if (s->dv.total_tokens > 0 && (!q || !k || !v || !out)) return RSWA_EINVAL;
+  if (s->dv.total_tokens > 0 &&
+      (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
+    return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = launch_cache_fill(s->dv, k, v, s->k_cache[(size_t)layer], s->v_cache[(size_t)layer], st);
+  if (e == cudaSuccess) {
+    e = launch_prefill_simt(s->dv, q, k, v, out, st);
+  }
+  if (e != cudaSuccess) return RSWA_ECUDA;
+  s->layer_ready[(size_t)layer] = 1;
+  return RSWA_OK;
+}
+
+rswa_status rswa_decode_step(rswa_state *s, int32_t layer, const void *q, const void *k_new,
+                             const void *v_new, void *out, void *stream) {
+  if (!s || layer < 0 || layer >= s->cfg.num_layers) return RSWA_EINVAL;
+  if (!q || !k_new || !v_new || !out) return RSWA_EINVAL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out))
+    return RSWA_EINVAL;
+  if (!s->layer_ready[(size_t)layer]) return RSWA_ESTATE;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  return from_cuda(launch_decode(s->dv, q, k_new, v_new, s->k_cache[(size_t)layer],
+                                 s->v_cache[(size_t)layer], out, (cudaStream_t)stream));
+}
+
+rswa_status rswa_advance(rswa_state *s, void *stream) {
+  if (!s) return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  return from_cuda(launch_advance(s->dv, (cudaStream_t)stream));
+}
+
+rswa_status rswa_reset_ring(rswa_state *s, void *stream) {
+  if (!s) return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  return from_cuda(cudaMemcpyAsync(s->dv.t, s->dv.t + s->cfg.batch,
+                                   (size_t)s->cfg.batch * sizeof(int64_t),
+                                   cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+}
+
+rswa_status rswa_ngram_mask(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                            const int32_t *hist_len, int32_t rows, int32_t vocab, int32_t n,
+                            int32_t window, int32_t *device_error, void *stream) {
+  if (rows < 0 || vocab < 1 || n < 1 || window < 0 || ld < vocab || hist_ld < window)
+    return RSWA_EINVAL;
+  if (rows > 0 && (!logits || (window > 0 && !history))) return RSWA_EINVAL;
+  if (rows == 0) return RSWA_OK;
+  return from_cuda(launch_ngram(logits, ld, history, hist_ld, hist_len, rows, vocab, n, window,
+                                device_error, (cudaStream_t)stream));
+}
+
+rswa_status rswa_get_ring(const rswa_state *s, int64_t *n_generated, int32_t *ring_pos,
+                          int64_t *cache_len, void *stream) {
+  if (!s) return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  std::vector<int64_t> t((size_t)s->cfg.batch);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(t.data(), s->dv.t, t.size() * sizeof(int64_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return RSWA_ECUDA;
+  const int64_t W = s->cfg.window;
+  for (int b = 0; b < s->cfg.batch; ++b) {
+    if (n_generated) n_generated[b] = t[(size_t)b];
+    if (ring_pos) ring_pos[b] = (int32_t)(t[(size_t)b] < W ? 0 : t[(size_t)b] % W);
+    if (cache_len) cache_len[b] = s->plen[(size_t)b] + std::min(t[(size_t)b], W);
+  }
+  return RSWA_OK;
+}
+
+rswa_status rswa_check_device_error(rswa_state *s, void *stream) {
+  if (!s) return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  int word = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&word, s->dv.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(s->dv.err, 0, sizeof(int));
+  if (e != cudaSuccess) return RSWA_ECUDA;
+  if (word & RSWA_DEVERR_TIMEOUT) return RSWA_ETIMEOUT;
+  if (word) return RSWA_EDEVICE;
+  return RSWA_OK;
+}
+
+const char *rswa_status_string(rswa_status st) {
+  switch (st) {
+    case RSWA_OK: return "ok";
+    case RSWA_EINVAL: return "invalid argument";
+    case RSWA_ENOMEM: return "workspace too small";
+    case RSWA_ECUDA: return "CUDA call or kernel launch failed";
+    case RSWA_ESTATE: return "call out of order (layer not prefilled)";
+    case RSWA_ETIMEOUT: return "a kernel's bounded wait ran out";
+    case RSWA_EDEVICE: return "a kernel rejected its data";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

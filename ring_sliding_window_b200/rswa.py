@@ -1,0 +1,245 @@
+"""Thin ctypes binding of librswa (include/rswa.h), same names as the C ABI.
+
+Functions here only marshal arguments: torch tensors become raw device
+pointers, the current torch CUDA stream becomes the ``stream`` argument, and a
+non-zero status becomes an ``RswaError``.  All computation happens in the CUDA
+kernels of librswa.so; if that library is missing this module raises at import.
+
+``State`` is a convenience owner of the device memory a batch needs (one K and
+one V cache per layer, and the workspace), allocated through torch, plus the
+opaque ``rswa_state``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "librswa.so")
+
+RSWA_OK, RSWA_EINVAL, RSWA_ENOMEM, RSWA_ECUDA, RSWA_ESTATE, RSWA_ETIMEOUT, RSWA_EDEVICE = range(7)
+RSWA_F32, RSWA_BF16 = 0, 1
+RSWA_DEVERR_TIMEOUT, RSWA_DEVERR_BAD_TOKEN, RSWA_DEVERR_BAD_LENGTH = 1, 2, 4
+
+EXPORTED = (
+    "rswa_cache_bytes", "rswa_workspace_bytes", "rswa_state_create", "rswa_state_destroy",
+    "rswa_cache_offset", "rswa_prefill", "rswa_decode_step", "rswa_advance", "rswa_reset_ring",
+    "rswa_ngram_mask", "rswa_get_ring", "rswa_check_device_error", "rswa_status_string",
+)
+
+
+class RswaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class rswa_config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_layers", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"librswa.so is missing at {_LIB_PATH}; build it with "
+                      "`python -m ring_sliding_window_b200.build` (needs nvcc)")
+
+lib = ctypes.CDLL(_LIB_PATH)
+
+_vp = ctypes.c_void_p
+_cfgp = ctypes.POINTER(rswa_config)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+lib.rswa_cache_bytes.argtypes = [_cfgp, _i64p]
+lib.rswa_cache_bytes.restype = ctypes.c_size_t
+lib.rswa_workspace_bytes.argtypes = [_cfgp, _i64p]
+lib.rswa_workspace_bytes.restype = ctypes.c_size_t
+lib.rswa_state_create.argtypes = [_cfgp, _i64p, _i64p, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                  _vp, ctypes.c_size_t, _vp, ctypes.POINTER(_vp)]
+lib.rswa_state_destroy.argtypes = [_vp]
+lib.rswa_cache_offset.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64]
+lib.rswa_cache_offset.restype = ctypes.c_int64
+lib.rswa_prefill.argtypes = [_vp, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
+lib.rswa_decode_step.argtypes = [_vp, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
+lib.rswa_advance.argtypes = [_vp, _vp]
+lib.rswa_reset_ring.argtypes = [_vp, _vp]
+lib.rswa_ngram_mask.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, ctypes.c_int32,
+                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp]
+lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
+lib.rswa_check_device_error.argtypes = [_vp, _vp]
+lib.rswa_status_string.argtypes = [ctypes.c_int]
+lib.rswa_status_string.restype = ctypes.c_char_p
+for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_decode_step",
+           "rswa_advance", "rswa_reset_ring", "rswa_ngram_mask", "rswa_get_ring",
+           "rswa_check_device_error"):
+    getattr(lib, _n).restype = ctypes.c_int
+
+
+def status_string(status: int) -> str:
+    return lib.rswa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != RSWA_OK:
+        raise RswaError(status, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _i64(vals: Sequence[int]):
+    return (ctypes.c_int64 * len(vals))(*[int(x) for x in vals])
+
+
+def make_config(batch, num_layers, num_heads, head_dim, window, dtype, scale=0.0) -> rswa_config:
+    d = RSWA_BF16 if dtype in (torch.bfloat16, RSWA_BF16, "bf16") else RSWA_F32
+    return rswa_config(batch, num_layers, num_heads, head_dim, window, d, float(scale))
+
+
+# ----------------------------------------------------------------- C names
+def rswa_cache_bytes(cfg: rswa_config, prefill_len: Sequence[int]) -> int:
+    return int(lib.rswa_cache_bytes(ctypes.byref(cfg), _i64(prefill_len)))
+
+
+def rswa_workspace_bytes(cfg: rswa_config, prefill_len: Sequence[int]) -> int:
+    return int(lib.rswa_workspace_bytes(ctypes.byref(cfg), _i64(prefill_len)))
+
+
+def rswa_state_create(cfg, prefill_len, n_generated, k_cache, v_cache, workspace,
+                      workspace_size, stream=None) -> ctypes.c_void_p:
+    kp = (ctypes.c_void_p * len(k_cache))(*[_ptr(t).value for t in k_cache])
+    vp = (ctypes.c_void_p * len(v_cache))(*[_ptr(t).value for t in v_cache])
+    out = ctypes.c_void_p()
+    st = lib.rswa_state_create(ctypes.byref(cfg), _i64(prefill_len),
+                               None if n_generated is None else _i64(n_generated), kp, vp,
+                               _ptr(workspace), int(workspace_size), _stream(stream),
+                               ctypes.byref(out))
+    _check(st, "rswa_state_create")
+    return out
+
+
+def rswa_state_destroy(state) -> None:
+    _check(lib.rswa_state_destroy(state), "rswa_state_destroy")
+
+
+def rswa_cache_offset(state, b: int, h: int, slot: int) -> int:
+    return int(lib.rswa_cache_offset(state, b, h, slot))
+
+
+def rswa_prefill(state, layer, q, k, v, out, stream=None) -> None:
+    _check(lib.rswa_prefill(state, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream)),
+           "rswa_prefill")
+
+
+def rswa_decode_step(state, layer, q, k_new, v_new, out, stream=None) -> None:
+    _check(lib.rswa_decode_step(state, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                _stream(stream)), "rswa_decode_step")
+
+
+def rswa_advance(state, stream=None) -> None:
+    _check(lib.rswa_advance(state, _stream(stream)), "rswa_advance")
+
+
+def rswa_reset_ring(state, stream=None) -> None:
+    _check(lib.rswa_reset_ring(state, _stream(stream)), "rswa_reset_ring")
+
+
+def rswa_ngram_mask(logits, history, hist_len, n: int, window: int, device_error=None,
+                    stream=None, vocab: Optional[int] = None) -> None:
+    """logits: cuda float32 [rows, ld]; history: cuda int32 [rows, hist_ld]."""
+    rows = logits.shape[0]
+    ld = logits.stride(0) if rows else logits.shape[1]
+    vocab = logits.shape[1] if vocab is None else vocab
+    hist_ld = history.stride(0) if rows else window
+    _check(lib.rswa_ngram_mask(_ptr(logits), ld, _ptr(history), hist_ld, _ptr(hist_len), rows,
+                               vocab, n, window, _ptr(device_error), _stream(stream)),
+           "rswa_ngram_mask")
+
+
+def rswa_get_ring(state, batch: int, stream=None):
+    """Returns (n_generated[B], ring_pos[B], cache_len[B]) as Python lists."""
+    n = (ctypes.c_int64 * batch)()
+    rp = (ctypes.c_int32 * batch)()
+    cl = (ctypes.c_int64 * batch)()
+    _check(lib.rswa_get_ring(state, n, rp, cl, _stream(stream)), "rswa_get_ring")
+    return list(n), list(rp), list(cl)
+
+
+def rswa_check_device_error(state, stream=None) -> int:
+    """Returns the status (does not raise): RSWA_OK, RSWA_ETIMEOUT or RSWA_EDEVICE."""
+    return int(lib.rswa_check_device_error(state, _stream(stream)))
+
+
+# ---------------------------------------------------------- owning helper
+class State:
+    """A batch's caches + workspace (torch-allocated) and its rswa_state."""
+
+    def __init__(self, batch, num_layers, num_heads, head_dim, window, prefill_lens,
+                 dtype=torch.bfloat16, n_generated=None, scale=0.0, device="cuda", stream=None):
+        self.cfg = make_config(batch, num_layers, num_heads, head_dim, window, dtype, scale)
+        self.dtype = torch.bfloat16 if self.cfg.dtype == RSWA_BF16 else torch.float32
+        self.prefill_lens = [int(p) for p in prefill_lens]
+        self.B, self.L, self.H, self.d, self.W = batch, num_layers, num_heads, head_dim, window
+        cb = rswa_cache_bytes(self.cfg, self.prefill_lens)
+        wb = rswa_workspace_bytes(self.cfg, self.prefill_lens)
+        if cb == 0 or wb == 0:
+            raise RswaError(RSWA_EINVAL, "rswa_cache_bytes/rswa_workspace_bytes")
+        elems = cb // (2 if self.dtype == torch.bfloat16 else 4)
+        self.k_cache = [torch.empty(elems, dtype=self.dtype, device=device) for _ in range(num_layers)]
+        self.v_cache = [torch.empty(elems, dtype=self.dtype, device=device) for _ in range(num_layers)]
+        self.workspace = torch.empty(wb, dtype=torch.uint8, device=device)
+        self.handle = rswa_state_create(self.cfg, self.prefill_lens, n_generated, self.k_cache,
+                                        self.v_cache, self.workspace, wb, stream)
+
+    def close(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h:
+            rswa_state_destroy(h)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def cache_view(self, layer: int, which: str, b: int, h: int) -> torch.Tensor:
+        """[P_b + W, d] view of one (b, h) ring of a layer's K or V cache."""
+        off = rswa_cache_offset(self.handle, b, h, 0)
+        n = (self.prefill_lens[b] + self.W) * self.d
+        buf = (self.k_cache if which == "k" else self.v_cache)[layer]
+        return buf[off:off + n].view(self.prefill_lens[b] + self.W, self.d)
+
+    def prefill(self, layer, q, k, v, out, stream=None):
+        rswa_prefill(self.handle, layer, q, k, v, out, stream)
+
+    def decode_step(self, layer, q, k_new, v_new, out, stream=None):
+        rswa_decode_step(self.handle, layer, q, k_new, v_new, out, stream)
+
+    def advance(self, stream=None):
+        rswa_advance(self.handle, stream)
+
+    def reset_ring(self, stream=None):
+        rswa_reset_ring(self.handle, stream)
+
+    def ring(self, stream=None):
+        return rswa_get_ring(self.handle, self.B, stream)
+
+    def check(self, stream=None) -> int:
+        return rswa_check_device_error(self.handle, stream)
