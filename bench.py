@@ -339,9 +339,17 @@ def cpu_oracle_rate(w: synth.Workload, seconds: float, max_steps=None, layers_pe
 
 
 # --------------------------------------------------------------------------
+def _workload(args):
+    import dataclasses
+    w = synth.workload(args.workload)
+    if args.layers:
+        w = dataclasses.replace(w, layers=args.layers)
+    return w
+
+
 def run_ours(args, rank, world, local_rank):
     hbm_peak, tc_peak, peak_src = measured_peaks()
-    w = synth.workload(args.workload)
+    w = _workload(args)
     dev = torch.cuda.current_device()
     s = torch.cuda.Stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -464,7 +472,7 @@ def run_also(w, args, flush, s, hbm_peak, tc_peak):
 
 
 def run_reference(args):
-    w = synth.workload(args.workload)
+    w = _workload(args)
     # size the sample: measure one step, then choose layers per step so that
     # warmup + steps fit in the time budget
     rate1, _, el1, _, _ = cpu_oracle_rate(w, 0.0, max_steps=1, layers_per_step=1)
@@ -496,6 +504,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="single_page_decode")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (small profiling runs)")
     ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving")
     ap.add_argument("--also-steps", type=int, default=40)
     ap.add_argument("--skip-prefill-also", action="store_true")
