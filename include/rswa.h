@@ -197,6 +197,44 @@ rswa_status rswa_check_device_error(rswa_state *state, void *stream);
 /* Static description of a status code. */
 const char *rswa_status_string(rswa_status status);
 
+/* ---- Allocation-free decode step --------------------------------------
+ * This call has no counterpart in the paper; it exists for callers that
+ * cannot hand the library a workspace.  A plugin hosted by another runtime
+ * or inference server gets its input and output tensors but may not allocate
+ * device memory itself (the host application's allocator owns the pool, so a
+ * private cudaMalloc can fail or fragment it), and a latency-bound serving
+ * loop keeps cudaMalloc/cudaFree off its hot path because both can
+ * synchronise the device.
+ *
+ * Same computation as rswa_decode_step for ONE layer, without a state: the
+ * caller passes the ring position explicitly and advances it itself.
+ *  cfg           : as for rswa_state_create (num_layers is ignored).
+ *  prefill_len   : host [B], P_b.
+ *  n_generated   : host [B], t_b = tokens generated before this step; the
+ *                  step writes slot P_b + (t_b mod W) and attends over
+ *                  slots [0, P_b + min(t_b + 1, W)).
+ *  k_cache, v_cache : device, this layer's caches in the layout above.
+ *  q, k_new, v_new, out : device [B][H][d].  All device pointers 16-byte aligned.
+ *  device_error  : device int32 or NULL; kernel error bits are ORed into it
+ *                  (NULL: they go to a word inside the scratch, cleared by
+ *                  each call, and are not reported).
+ * Scratch: a file-scope device array of RSWA_NOALLOC_SCRATCH_BYTES bytes on
+ * every device that loads the library, held until the process exits.  The
+ * call allocates nothing (no cudaMalloc/cudaFree).  Its first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture.  The work tables are copied into
+ * the array from pageable host memory on `stream` at every call.  Every call
+ * on a device shares the one array and it keeps the last call's contents, so
+ * calls whose work overlaps on the GPU (different streams, no ordering)
+ * race and corrupt each other; order them on one stream.
+ * Returns RSWA_EINVAL for bad arguments and RSWA_ENOMEM when the batch needs
+ * more scratch than the array holds (rswa_workspace_bytes() > the limit). */
+#define RSWA_NOALLOC_SCRATCH_BYTES (4u << 20)
+rswa_status rswa_decode_step_noalloc(const rswa_config *cfg, const int64_t *prefill_len,
+                                     const int64_t *n_generated, void *k_cache, void *v_cache,
+                                     const void *q, const void *k_new, const void *v_new,
+                                     void *out, int32_t *device_error, void *stream);
+
 /* Bits of a device error word. */
 #define RSWA_DEVERR_TIMEOUT 1
 #define RSWA_DEVERR_BAD_TOKEN 2

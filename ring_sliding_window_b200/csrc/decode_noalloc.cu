@@ -1,0 +1,129 @@
+// Allocation-free variant of the decode step.
+//
+// rswa_decode_step needs a caller-allocated workspace (work tables, ring
+// counters and the split-K partials).  Some callers cannot provide one at the
+// point where they decode: a plugin hosted by another runtime or inference
+// server receives its input and output tensors but must not allocate device
+// memory itself (the host application's allocator already owns the pool, so a
+// private cudaMalloc can fail or fragment it), and a latency-bound serving
+// loop must keep cudaMalloc/cudaFree off its hot path because both can
+// synchronise the device and stall every other stream.
+//
+// rswa_decode_step_noalloc serves them: it runs the same split-K kernels as
+// rswa_decode_step, with the scratch taken from a file-scope __device__ array
+// of a fixed size (kNoAllocScratchBytes per device, held until the process
+// exits).  The caller still passes the cache, inputs and outputs.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace rswa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = RSWA_NOALLOC_SCRATCH_BYTES;
+
+// Shared by every call on a device.  Host code must not use this name as an
+// address: the device address comes from cudaGetSymbolAddress below.
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mu;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array for `dev` (the current device), looked
+// up once per device.
+rswa_status scratch_for_device(int dev, uint8_t **out) {
+  if (dev < 0 || dev >= kMaxDevices) return RSWA_EINVAL;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (!g_scratch_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RSWA_ECUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = (uint8_t *)g_scratch_ptr[dev];
+  return RSWA_OK;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+}  // namespace rswa
+
+using namespace rswa;
+
+extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
+                                                const int64_t *prefill_len,
+                                                const int64_t *n_generated, void *k_cache,
+                                                void *v_cache, const void *q, const void *k_new,
+                                                const void *v_new, void *out,
+                                                int32_t *device_error, void *stream) {
+  if (!config_ok(cfg, prefill_len) || !n_generated) return RSWA_EINVAL;
+  if (!k_cache || !v_cache || !q || !k_new || !v_new || !out) return RSWA_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(k_new) ||
+      !aligned16(v_new) || !aligned16(out))
+    return RSWA_EINVAL;
+  const int B = cfg->batch;
+  for (int b = 0; b < B; ++b)
+    if (n_generated[b] < 0) return RSWA_EINVAL;
+  const int dev = current_device();
+  if (dev < 0) return RSWA_ECUDA;
+
+  const DecodePlan plan =
+      plan_decode(cfg, prefill_len, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+  const WsLayout ws = layout_ws(cfg, plan);
+  if (ws.total > kNoAllocScratchBytes) return RSWA_ENOMEM;  // batch too large for the array
+
+  uint8_t *scratch = nullptr;
+  const rswa_status st = scratch_for_device(dev, &scratch);
+  if (st != RSWA_OK) return st;
+
+  // Host image of the tables.  The error word at its head is zero, so every
+  // call starts from a cleared word; the partials are fully overwritten by
+  // the split kernel and need no clearing.
+  std::vector<uint8_t> img(ws.part_ml, 0);
+  int64_t *t = (int64_t *)(img.data() + ws.t);
+  int32_t *pl = (int32_t *)(img.data() + ws.plen);
+  int64_t *sb = (int64_t *)(img.data() + ws.slot_base);
+  for (int b = 0; b < B; ++b) {
+    t[b] = n_generated[b];
+    t[B + b] = n_generated[b];
+    pl[b] = (int32_t)prefill_len[b];
+    sb[b + 1] = sb[b] + prefill_len[b] + cfg->window;
+  }
+  memcpy(img.data() + ws.pieces, plan.pieces.data(), plan.pieces.size() * sizeof(DecodePiece));
+  memcpy(img.data() + ws.cta_piece, plan.cta_piece.data(), plan.cta_piece.size() * sizeof(int32_t));
+  memcpy(img.data() + ws.bh_piece, plan.bh_piece.data(), plan.bh_piece.size() * sizeof(int32_t));
+  cudaStream_t s = (cudaStream_t)stream;
+  // Pageable source: the call returns once the bytes are staged, so `img`
+  // may go out of scope; the copy is ordered before the kernels on `s`.
+  if (cudaMemcpyAsync(scratch, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RSWA_ECUDA;
+
+  DeviceView v;
+  memset(&v, 0, sizeof(v));
+  v.B = B;
+  v.H = cfg->num_heads;
+  v.D = cfg->head_dim;
+  v.W = cfg->window;
+  v.L = 1;
+  v.dtype = cfg->dtype;
+  v.scale = cfg->scale == 0.f ? 1.0f / sqrtf((float)cfg->head_dim) : cfg->scale;
+  v.err = device_error ? (int *)device_error : (int *)(scratch + ws.err);
+  v.t = (int64_t *)(scratch + ws.t);
+  v.plen = (const int32_t *)(scratch + ws.plen);
+  v.slot_base = (const int64_t *)(scratch + ws.slot_base);
+  v.pieces = (const DecodePiece *)(scratch + ws.pieces);
+  v.cta_piece = (const int32_t *)(scratch + ws.cta_piece);
+  v.bh_piece = (const int32_t *)(scratch + ws.bh_piece);
+  v.part_ml = (float2 *)(scratch + ws.part_ml);
+  v.part_o = (float *)(scratch + ws.part_o);
+  v.decode_grid = plan.grid;
+  v.n_pieces = plan.n_pieces;
+  return launch_decode(v, q, k_new, v_new, k_cache, v_cache, out, s) == cudaSuccess ? RSWA_OK
+                                                                                     : RSWA_ECUDA;
+}

@@ -110,4 +110,11 @@ cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int6
 // Resident decode CTAs per SM for (dtype, head_dim); used by the planner.
 int decode_ctas_per_sm(int dtype, int head_dim);
 
+// Host-side helpers of the planner (rswa_api.cu).
+bool config_ok(const rswa_config *c, const int64_t *plen);
+int current_device();
+int sm_count(int dev);
+DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, int ctas_per_sm);
+WsLayout layout_ws(const rswa_config *c, const DecodePlan &p);
+
 }  // namespace rswa

@@ -13,8 +13,10 @@
 using namespace rswa;
 
 namespace {
-
 constexpr int64_t kMinRowsPerCta = 64;  // below this a decode CTA is mostly latency
+}  // namespace
+
+namespace rswa {
 
 bool config_ok(const rswa_config *c, const int64_t *plen) {
   if (!c || !plen) return false;
@@ -31,9 +33,17 @@ bool config_ok(const rswa_config *c, const int64_t *plen) {
   return true;
 }
 
+}  // namespace rswa
+
+namespace {
+
 size_t elem_size(const rswa_config *c) { return c->dtype == RSWA_BF16 ? 2 : 4; }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+namespace rswa {
 
 int current_device() {
   int d = -1;
@@ -112,6 +122,10 @@ WsLayout layout_ws(const rswa_config *c, const DecodePlan &p) {
   w.total = off;
   return w;
 }
+
+}  // namespace rswa
+
+namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 

@@ -28,7 +28,9 @@ EXPORTED = (
     "rswa_cache_bytes", "rswa_workspace_bytes", "rswa_state_create", "rswa_state_destroy",
     "rswa_cache_offset", "rswa_prefill", "rswa_decode_step", "rswa_advance", "rswa_reset_ring",
     "rswa_ngram_mask", "rswa_get_ring", "rswa_check_device_error", "rswa_status_string",
+    "rswa_decode_step_noalloc",
 )
+RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class RswaError(RuntimeError):
@@ -71,6 +73,8 @@ lib.rswa_ngram_mask.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, c
                                 ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp]
 lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
+lib.rswa_decode_step_noalloc.argtypes = [_cfgp, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.rswa_decode_step_noalloc.restype = ctypes.c_int
 lib.rswa_status_string.argtypes = [ctypes.c_int]
 lib.rswa_status_string.restype = ctypes.c_char_p
 for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_decode_step",
@@ -185,6 +189,16 @@ def rswa_get_ring(state, batch: int, stream=None):
 def rswa_check_device_error(state, stream=None) -> int:
     """Returns the status (does not raise): RSWA_OK, RSWA_ETIMEOUT or RSWA_EDEVICE."""
     return int(lib.rswa_check_device_error(state, _stream(stream)))
+
+
+def rswa_decode_step_noalloc(cfg: rswa_config, prefill_len, n_generated, k_cache, v_cache,
+                             q, k_new, v_new, out, device_error=None, stream=None) -> None:
+    """One layer's decode step with scratch in the library's static device array
+    (for callers that cannot allocate a workspace); t_b passed explicitly."""
+    _check(lib.rswa_decode_step_noalloc(ctypes.byref(cfg), _i64(prefill_len), _i64(n_generated),
+                                        _ptr(k_cache), _ptr(v_cache), _ptr(q), _ptr(k_new),
+                                        _ptr(v_new), _ptr(out), _ptr(device_error),
+                                        _stream(stream)), "rswa_decode_step_noalloc")
 
 
 # ---------------------------------------------------------- owning helper
