@@ -200,7 +200,7 @@ class DecodeRig:
         torch.cuda.synchronize()
 
     def launches_per_token(self):
-        return 2 * self.w.layers + 2
+        return self.w.layers + 2  # one decode kernel per layer, advance, n-gram mask
 
     def ring_t(self):
         n, _, _ = self.st.ring(stream=self.s)
@@ -242,23 +242,33 @@ def timed_tokens(rig: DecodeRig, steps: int, warmup: int, flush, sampler=None):
     return ms, ts, clocks
 
 
-def timed_decode_launches(rig: DecodeRig, n: int, flush):
-    """Eager rswa_decode_step launches (split-K + combine), each bracketed by
-    events after an L2 flush that keeps the GPU busy while the CPU enqueues."""
+def timed_decode_launches(rig: DecodeRig, reps: int, flush):
+    """Average duration of one decode_split_kernel launch (one rswa_decode_step)
+    in the bench's launch configuration: a CUDA graph of the layers' decode
+    steps only (no advance, so every replay sees the same ring position),
+    replayed after an L2 flush and bracketed by events on the stream; the
+    replay time divided by the layer count."""
     w, s = rig.w, rig.s
-    evs = []
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for l in range(w.layers):
+            rig.st.decode_step(l, rig.q[l], rig.kn[l], rig.vn[l], rig.out[l], stream=s)
+    torch.cuda.synchronize()
     t0 = rig.ring_t()
+    evs = []
     with torch.cuda.stream(s):
-        for i in range(n):
-            l = i % w.layers
+        g.replay()
+        for _ in range(reps):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(s)
-            rig.st.decode_step(l, rig.q[l], rig.kn[l], rig.vn[l], rig.out[l], stream=s)
+            g.replay()
             e1.record(s)
             evs.append((e0, e1))
     s.synchronize()
-    ms = [a.elapsed_time(b) for a, b in evs]
+    ms = [a.elapsed_time(b) / w.layers for a, b in evs]
+    del g
     return ms, t0
 
 
@@ -371,8 +381,8 @@ def run_ours(args, rank, world, local_rank):
     kv_bytes = sum(w.layers * kv_bytes_per_layer(w, t) for t in ts)
     kv_gbs = kv_bytes / (sum(ms) / 1e3) / 1e9
 
-    # ---- dominant kernel: rswa_decode_step (split-K + combine), eager launches
-    launch_ms, t_at = timed_decode_launches(rig, max(24, 2 * w.layers), flush)
+    # ---- dominant kernel: decode_split_kernel (one per rswa_decode_step)
+    launch_ms, t_at = timed_decode_launches(rig, 16, flush)
     per_launch_bytes = kv_bytes_per_layer(w, t_at)
     dur = statistics.mean(launch_ms) / 1e3
     achieved = per_launch_bytes / dur / 1e9
@@ -406,7 +416,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
                    "parallelism": f"replicas x{world}"},
         "kv_read_gbs": kv_gbs,
-        "roofline": {"kernel": "rswa_decode_step (decode_split_kernel + decode_combine_kernel)",
+        "roofline": {"kernel": "decode_split_kernel (rswa_decode_step: ring write + split-K "
+                               "attention + in-kernel combine)",
                      "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_source": peak_src,
                      "frac_of_datasheet_8000": achieved / DATASHEET_HBM_GBS,
@@ -418,7 +429,7 @@ def run_ours(args, rank, world, local_rank):
                     "ms_per_layer": pf_mean * 1e3, "flops_per_layer": pf_flops},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * (2 * w.layers + 2),
+        "gpu_launches": args.steps * (w.layers + 2),
         "clocks": clocks,
     }
 
@@ -445,7 +456,7 @@ def run_also(w, args, flush, s, hbm_peak, tc_peak):
     rig.capture()
     ms, ts, _ = timed_tokens(rig, steps, args.warmup, flush)
     kv_bytes = sum(w.layers * kv_bytes_per_layer(w, t) for t in ts)
-    launch_ms, t_at = timed_decode_launches(rig, 2 * w.layers, flush)
+    launch_ms, t_at = timed_decode_launches(rig, 8, flush)
     per_launch = kv_bytes_per_layer(w, t_at)
     ach = per_launch / (statistics.mean(launch_ms) / 1e3) / 1e9
     res = {"workload": w.name, "decode_steps_per_s": steps / (sum(ms) / 1e3),

@@ -21,8 +21,11 @@
 //  - The CTA whose piece holds this step's write slot stores k_new/v_new to
 //    the cache and substitutes them for that row from shared memory, so no CTA
 //    ever uses the stale slot and nobody re-reads the fresh one.
-//  - Each piece ends in an unnormalised partial (m, l, o[d]); the combine
-//    kernel merges the pieces of each (b, h).
+//  - Each piece ends in an unnormalised partial (m, l, o[d]) in the
+//    workspace.  The CTA that finishes the last piece of a (b, h) (a counter
+//    per (b, h), bumped after a release fence) merges that ring's partials by
+//    log-sum-exp and writes the output, then re-arms the counter: the combine
+//    pass runs inside the same launch, overlapped with other CTAs' streaming.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -34,6 +37,7 @@ namespace rswa {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMergeBatch = 16;  // partials whose loads are in flight together in the merge
 
 template <typename T, int D>
 struct DecodeShape {
@@ -63,6 +67,7 @@ struct __align__(128) DecodeSmem {
   float red_o[S::kGroups][D];
   float red_m[S::kGroups];
   float red_l[S::kGroups];
+  int is_last;
   uint64_t full[S::kStages];
   uint64_t empty[S::kStages];
 };
@@ -71,6 +76,7 @@ struct DecodeArgs {
   DeviceView v;
   const void *q, *k_new, *v_new;
   void *kc, *vc;
+  void *out;
 };
 
 __device__ __forceinline__ int64_t seg_offset_rows(const DeviceView &v, int b, int h, int plen) {
@@ -99,6 +105,12 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     fence_mbar_init();
   }
   __syncthreads();
+  // Everything above touched only this launch's shared memory and the work
+  // tables written when the state was built; from here on the kernel reads
+  // q/k_new/v_new, the ring counters and the cache, which earlier kernels in
+  // the stream may still be producing.
+  grid_dependency_wait();
+  allow_dependents();
 
   if (warp == S::kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -284,40 +296,66 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         for (int gg = 0; gg < S::kGroups; ++gg) L = fmaf(sm.red_l[gg], exp2f(sm.red_m[gg] - M), L);
       v.part_ml[p] = make_float2(M, L);
     }
+    // -------- publish the partial; the last piece of this (b, h) merges
+    __threadfence();
     named_bar_sync(1, 128);
-  }
-}
-
-template <typename T, int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DeviceView v, T *out) {
-  const int bh = blockIdx.x;
-  const int e = threadIdx.x;
-  const int p0 = v.bh_piece[bh], p1 = v.bh_piece[bh + 1];
-  float M = -INFINITY;
-  for (int p = p0; p < p1; ++p) {
-    const float2 ml = v.part_ml[p];
-    if (ml.y > 0.f) M = fmaxf(M, ml.x);
-  }
-  float L = 0.f, acc = 0.f;
-  for (int p = p0; p < p1; ++p) {
-    const float2 ml = v.part_ml[p];
-    if (ml.y > 0.f) {
-      const float w = exp2f(ml.x - M);
-      L = fmaf(w, ml.y, L);
-      acc = fmaf(w, v.part_o[(int64_t)p * D + e], acc);
+    const int p0 = v.bh_piece[pc.bh], np = v.bh_piece[pc.bh + 1] - p0;
+    if (tid == 0) {
+      int last = 1;
+      if (np > 1) {
+        last = atomicAdd(&v.bh_count[pc.bh], 1) == np - 1;
+        if (last) v.bh_count[pc.bh] = 0;  // re-arm for the next launch
+      }
+      sm.is_last = last;
+    }
+    named_bar_sync(1, 128);
+    if (sm.is_last) {
+      __threadfence();
+      // Thread tid merges output element tid.  Partials are read straight
+      // from L2, kMergeBatch at a time with every load of a batch in flight
+      // together, merged online by log-sum-exp.
+      float Mg = -INFINITY, Lg = 0.f, acc = 0.f;
+      for (int c0 = 0; c0 < np; c0 += kMergeBatch) {
+        float2 ml[kMergeBatch];
+        float ov[kMergeBatch];
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) {
+          const bool ok = c0 + i < np;
+          const int64_t pp = p0 + c0 + i;
+          ml[i] = ok ? __ldcg(&v.part_ml[pp]) : make_float2(-INFINITY, 0.f);
+          ov[i] = (ok && tid < D) ? __ldcg(&v.part_o[pp * D + tid]) : 0.f;
+        }
+        float Mc = Mg;
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) Mc = fmaxf(Mc, ml[i].x);
+        if (Mc == -INFINITY) continue;
+        const float corr = exp2f(Mg - Mc);
+        Lg *= corr;
+        acc *= corr;
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) {
+          const float wgt = exp2f(ml[i].x - Mc);  // 0 for empty or absent pieces
+          Lg = fmaf(wgt, ml[i].y, Lg);
+          acc = fmaf(wgt, ov[i], acc);
+        }
+        Mg = Mc;
+      }
+      if (tid < D) ((T *)a.out)[(int64_t)pc.bh * D + tid] = from_float<T>(acc / Lg);
     }
   }
-  out[(int64_t)bh * D + e] = from_float<T>(acc / L);
 }
 
 __global__ void advance_kernel(int64_t *t, int B) {
+  grid_dependency_wait();  // the decode kernels before it read t
+  allow_dependents();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) t[b] += 1;
 }
 
 template <typename T, int D>
 cudaError_t launch_decode_t(const DeviceView &v, const void *q, const void *k_new,
-                            const void *v_new, void *kc, void *vc, void *out, cudaStream_t s) {
+                            const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
+                            bool pdl) {
   using S = DecodeShape<T, D>;
   const int smem = (int)sizeof(DecodeSmem<T, D>);
   static bool attr_set = false;  // per (T, D) instantiation
@@ -327,12 +365,18 @@ cudaError_t launch_decode_t(const DeviceView &v, const void *q, const void *k_ne
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  DecodeArgs a{v, q, k_new, v_new, kc, vc};
-  decode_split_kernel<T, D><<<v.decode_grid, S::kThreads, smem, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  decode_combine_kernel<T, D><<<v.B * v.H, D, 0, s>>>(v, (T *)out);
-  return cudaGetLastError();
+  DecodeArgs a{v, q, k_new, v_new, kc, vc, out};
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(v.decode_grid);
+  lc.blockDim = dim3(S::kThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, decode_split_kernel<T, D>, a);
 }
 
 template <typename T, int D>
@@ -353,19 +397,28 @@ int ctas_per_sm_t() {
 }  // namespace
 
 cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
-                          const void *v_new, void *kc, void *vc, void *out, cudaStream_t s) {
+                          const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
+                          bool pdl) {
   if (v.dtype == RSWA_BF16) {
     if (v.D == 128)
-      return launch_decode_t<__nv_bfloat16, 128>(v, q, k_new, v_new, kc, vc, out, s);
-    return launch_decode_t<__nv_bfloat16, 64>(v, q, k_new, v_new, kc, vc, out, s);
+      return launch_decode_t<__nv_bfloat16, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+    return launch_decode_t<__nv_bfloat16, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
   }
-  if (v.D == 128) return launch_decode_t<float, 128>(v, q, k_new, v_new, kc, vc, out, s);
-  return launch_decode_t<float, 64>(v, q, k_new, v_new, kc, vc, out, s);
+  if (v.D == 128) return launch_decode_t<float, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+  return launch_decode_t<float, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
 }
 
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s) {
-  advance_kernel<<<(v.B + 255) / 256, 256, 0, s>>>(v.t, v.B);
-  return cudaGetLastError();
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((v.B + 255) / 256);
+  lc.blockDim = dim3(256);
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, advance_kernel, v.t, v.B);
 }
 
 int decode_ctas_per_sm(int dtype, int head_dim) {

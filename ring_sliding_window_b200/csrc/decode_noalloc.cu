@@ -75,16 +75,16 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
 
   const DecodePlan plan =
       plan_decode(cfg, prefill_len, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
-  const WsLayout ws = layout_ws(cfg, plan);
+  const WsLayout ws = layout_ws(cfg, prefill_len, plan);
   if (ws.total > kNoAllocScratchBytes) return RSWA_ENOMEM;  // batch too large for the array
 
   uint8_t *scratch = nullptr;
   const rswa_status st = scratch_for_device(dev, &scratch);
   if (st != RSWA_OK) return st;
 
-  // Host image of the tables.  The error word at its head is zero, so every
-  // call starts from a cleared word; the partials are fully overwritten by
-  // the split kernel and need no clearing.
+  // Host image of the tables.  The error word and the per-(b, h) completion
+  // counters in it are zero, so every call starts from cleared values; the
+  // partials are fully overwritten by the split kernel and need no clearing.
   std::vector<uint8_t> img(ws.part_ml, 0);
   int64_t *t = (int64_t *)(img.data() + ws.t);
   int32_t *pl = (int32_t *)(img.data() + ws.plen);
@@ -120,10 +120,14 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
   v.pieces = (const DecodePiece *)(scratch + ws.pieces);
   v.cta_piece = (const int32_t *)(scratch + ws.cta_piece);
   v.bh_piece = (const int32_t *)(scratch + ws.bh_piece);
+  v.bh_count = (int *)(scratch + ws.bh_count);
   v.part_ml = (float2 *)(scratch + ws.part_ml);
   v.part_o = (float *)(scratch + ws.part_o);
   v.decode_grid = plan.grid;
   v.n_pieces = plan.n_pieces;
-  return launch_decode(v, q, k_new, v_new, k_cache, v_cache, out, s) == cudaSuccess ? RSWA_OK
-                                                                                     : RSWA_ECUDA;
+  // Plain launch (no programmatic dependent launch): the table upload just
+  // before it must be complete when the kernel starts.
+  return launch_decode(v, q, k_new, v_new, k_cache, v_cache, out, s, false) == cudaSuccess
+             ? RSWA_OK
+             : RSWA_ECUDA;
 }

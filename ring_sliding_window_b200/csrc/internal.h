@@ -30,9 +30,11 @@ struct WsLayout {
   size_t tok_base;   // int64 [B+1] sum_{b'<b} P_b'
   size_t tile_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kPrefillTile)
   size_t tile64_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kSimtTile)
+  size_t pf_tiles;   // int2 [total_tiles] (b, query tile), longest first
   size_t pieces;     // DecodePiece [n_pieces]
   size_t cta_piece;  // int32 [G+1] first piece of each decode CTA
   size_t bh_piece;   // int32 [B*H+1] first piece of each (b, h)
+  size_t bh_count;   // int32 [B*H]   pieces of (b, h) finished in this launch
   size_t part_ml;    // float2 [n_pieces] (running max in log2 units, sum)
   size_t part_o;     // float [n_pieces][d] unnormalised outputs
   size_t total;
@@ -62,9 +64,11 @@ struct DeviceView {
   const int64_t *tok_base;
   const int32_t *tile_base;
   const int32_t *tile64_base;
+  const int2 *pf_tiles;
   const DecodePiece *pieces;
   const int32_t *cta_piece;
   const int32_t *bh_piece;
+  int *bh_count;
   float2 *part_ml;
   float *part_o;
   int decode_grid;
@@ -94,15 +98,18 @@ struct rswa_state {
 namespace rswa {
 
 // Launchers (return cudaGetLastError() of their launch).
+// pdl: launch with programmatic stream serialization (the kernel waits for
+// the previous kernel's completion before touching any produced data).
 cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
-                          const void *v_new, void *kc, void *vc, void *out, cudaStream_t s);
+                          const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
+                          bool pdl);
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s);
 cudaError_t launch_cache_fill(const DeviceView &v, const void *k, const void *vv, void *kc,
                               void *vc, cudaStream_t s);
 cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,
                                 const void *vv, void *out, cudaStream_t s);
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, cudaStream_t s);
+                              void *out, const int2 *tiles, cudaStream_t s);
 cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
                          const int32_t *hist_len, int rows, int vocab, int n, int window,
                          int *err, cudaStream_t s);
@@ -115,6 +122,6 @@ bool config_ok(const rswa_config *c, const int64_t *plen);
 int current_device();
 int sm_count(int dev);
 DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, int ctas_per_sm);
-WsLayout layout_ws(const rswa_config *c, const DecodePlan &p);
+WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &p);
 
 }  // namespace rswa

@@ -1,0 +1,372 @@
+// Prefill causal attention on the 5th-generation tensor cores (bf16, d = 128).
+//
+// Method ("开源5天Star破万之后：百度Unlimited-OCR的爆火路径复盘", §2.1): the
+// prefill segment keeps full attention -- every prompt token attends causally
+// to all earlier tokens of its prompt.  The page's section 三 notes that the
+// transformers path materialises the whole score matrix; here it is a
+// flash-style kernel that never leaves the chip with it.
+//
+// One CTA computes one 128-row query tile of one (sequence, head):
+//   warp 4      TMA producer: the Q tile once, then K and V tiles (128 keys x
+//               128 dims, bf16, 128-byte swizzle) into a 2-stage ring;
+//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into a TMEM buffer
+//               (two buffers, 128 fp32 columns each), then O += P_j V_j with
+//               P_j read from TMEM (it overwrites S_j's columns as bf16 pairs);
+//               also owns the TMEM allocation;
+//   warps 0-3   softmax: thread r owns query row r (TMEM lane r).  It loads its
+//               S row, masks the diagonal tile, runs the online softmax in the
+//               log2 domain and writes P back to TMEM.  O (TMEM, fp32) is only
+//               rescaled when a warp's running max grows by more than 2^8;
+//               otherwise the stale max keeps every p <= 256, exact in the end
+//               because l uses the same max.  The epilogue divides by l and
+//               stores bf16 rows.
+// Query tiles are ordered longest-first (causal work grows with the tile
+// index).  Every mbarrier wait is bounded; on a timeout the kernel records it,
+// stops issuing work, waits (bounded) for what is in flight, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace rswa {
+namespace {
+
+constexpr int kTile = 128;   // query rows and keys per tile
+constexpr int kD = 128;      // head dim
+constexpr int kStages = 2;   // K/V ring depth
+constexpr int kHalfBytes = kTile * 64 * 2;   // one 64-column swizzled half: 16 KB
+constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;    // S buffers at columns 0 and 128
+constexpr uint32_t kColO = 256;  // O accumulator
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct __align__(1024) PrefillSmem {
+  uint8_t q[kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint64_t q_full;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_bar;      // one phase per finished PV MMA
+  uint64_t o_final;    // the last PV MMA finished
+  uint64_t mma_done;   // everything the MMA thread issued finished
+  uint32_t tmem_base;
+  int dead;
+};
+
+struct PrefillTcArgs {
+  DeviceView v;
+  const int2 *tiles;  // (b, q_tile) longest-first
+  __nv_bfloat16 *out;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *err,
+                                         volatile int *dead) {
+  if (*dead) return false;
+  if (mbar_wait_bounded(bar, parity, err, RSWA_DEVERR_TIMEOUT)) return true;
+  *dead = 1;
+  return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const PrefillTcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // dynamic shared memory is only 16-byte aligned: round up to 1024 for the swizzle atoms
+  PrefillSmem &sm = *reinterpret_cast<PrefillSmem *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const DeviceView &v = a.v;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int tile_id = blockIdx.x / v.H;
+  const int h = blockIdx.x % v.H;
+  const int2 bt = a.tiles[tile_id];
+  const int b = bt.x, qt = bt.y;
+  const int P = v.plen[b];
+  const int tok0 = (int)v.tok_base[b];
+  const int n_kv = qt + 1;  // causal: key tiles 0..qt
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 4);
+    }
+    mbar_init(&sm.o_bar, 1);
+    mbar_init(&sm.o_final, 1);
+    mbar_init(&sm.mma_done, 1);
+    sm.dead = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = sm.tmem_base;
+  volatile int *dead = &sm.dead;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      const int xh = h * kD;
+      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+      tc::tma_load_2d(sm.q, &tm_q, xh, tok0 + qt * kTile, &sm.q_full);
+      tc::tma_load_2d(sm.q + kHalfBytes, &tm_q, xh + 64, tok0 + qt * kTile, &sm.q_full);
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % kStages;
+        const uint32_t par = ((j / kStages) & 1) ^ 1;
+        const int y = tok0 + j * kTile;
+        if (!wait_bar(&sm.k_empty[s], par, v.err, dead)) break;
+        mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
+        tc::tma_load_2d(sm.k[s], &tm_k, xh, y, &sm.k_full[s]);
+        tc::tma_load_2d(sm.k[s] + kHalfBytes, &tm_k, xh + 64, y, &sm.k_full[s]);
+        if (!wait_bar(&sm.v_empty[s], par, v.err, dead)) {
+          issued = j + 1;  // K of tile j is in flight
+          break;
+        }
+        mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
+        tc::tma_load_2d(sm.v[s], &tm_v, xh, y, &sm.v_full[s]);
+        tc::tma_load_2d(sm.v[s] + kHalfBytes, &tm_v, xh + 64, y, &sm.v_full[s]);
+        issued = j + 1;
+      }
+      // every load issued has landed before the CTA may exit (bounded)
+      mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / kStages) * kStages;  // last tile using stage s
+        const uint32_t par = (last / kStages) & 1;
+        mbar_wait_bounded(&sm.k_full[s], par, v.err, RSWA_DEVERR_TIMEOUT);
+        mbar_wait_bounded(&sm.v_full[s], par, v.err, RSWA_DEVERR_TIMEOUT);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kTile, kTile, false, false);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kTile, kD, false, true);
+      const uint32_t q_addr = smem_u32(sm.q);
+      if (wait_bar(&sm.q_full, 0, v.err, dead)) {
+        for (int j = 0; j <= n_kv; ++j) {
+          if (j < n_kv) {
+            // S_j = Q K_j^T
+            const int s = j % kStages;
+            if (!wait_bar(&sm.k_full[s], (j / kStages) & 1, v.err, dead)) break;
+            tc::fence_after_sync();
+            const uint32_t k_addr = smem_u32(sm.k[s]);
+            const uint32_t d_s = tbase + kColS + (uint32_t)(j & 1) * kTile;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint32_t off = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
+              tc::mma_ss(d_s, tc::sw128_desc(q_addr + off, 16, 1024),
+                         tc::sw128_desc(k_addr + off, 16, 1024), idesc_qk, kk > 0);
+            }
+            tc::commit(&sm.s_full[j & 1]);
+            tc::commit(&sm.k_empty[s]);
+          }
+          if (j >= 1) {
+            // O += P_{j-1} V_{j-1}
+            const int jp = j - 1;
+            const int s = jp % kStages;
+            if (!wait_bar(&sm.p_full[jp & 1], (jp >> 1) & 1, v.err, dead)) break;
+            if (!wait_bar(&sm.v_full[s], (jp / kStages) & 1, v.err, dead)) break;
+            tc::fence_after_sync();
+            const uint32_t v_addr = smem_u32(sm.v[s]);
+            const uint32_t p_tmem = tbase + kColS + (uint32_t)(jp & 1) * kTile;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              tc::mma_ts(tbase + kColO, p_tmem + (uint32_t)kk * 8,
+                         tc::sw128_desc(v_addr + (uint32_t)kk * 2048, kHalfBytes, 1024), idesc_pv,
+                         (jp > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc::commit(&sm.o_bar);
+            tc::commit(&sm.v_empty[s]);
+            if (jp == n_kv - 1) tc::commit(&sm.o_final);
+          }
+        }
+      }
+      tc::commit(&sm.mma_done);
+      mbar_wait_bounded(&sm.mma_done, 0, v.err, RSWA_DEVERR_TIMEOUT);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = warp * 32 + lane;  // query row inside the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float sl2 = v.scale * kLog2e;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int buf = j & 1;
+      ok = wait_bar(&sm.s_full[buf], (j >> 1) & 1, v.err, dead);
+      if (!ok) break;
+      tc::fence_after_sync();
+      const uint32_t t_s = tbase + lane_off + kColS + (uint32_t)buf * kTile;
+      float s[kTile];
+      tc::ld32(t_s + 0, reinterpret_cast<uint32_t *>(s));
+      tc::ld32(t_s + 32, reinterpret_cast<uint32_t *>(s) + 32);
+      tc::ld32(t_s + 64, reinterpret_cast<uint32_t *>(s) + 64);
+      tc::ld32(t_s + 96, reinterpret_cast<uint32_t *>(s) + 96);
+      tc::wait_ld();
+      if (j == qt) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (c > r) s[c] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, s[c]);
+      mx *= sl2;
+      const float m_new = fmaxf(m_run, mx);
+      const bool need = j > 0 && m_new > m_run + kRescaleThreshold;
+      const bool rescale = __any_sync(0xffffffffu, need);
+      float m_use = m_run, alpha = 1.f;
+      if (j == 0) {
+        m_use = m_new;
+      } else if (rescale) {
+        m_use = m_new;
+        alpha = tc::ex2(m_run - m_new);
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = tc::ex2(fmaf(s[64 * half + 2 * c], sl2, -m_use));
+          const float p1 = tc::ex2(fmaf(s[64 * half + 2 * c + 1], sl2, -m_use));
+          rs += p0 + p1;
+          pk[c] = tc::pack_bf16x2(p0, p1);
+        }
+        tc::st32(t_s + 32 * half, pk);
+      }
+      l_run = l_run * alpha + rs;
+      m_run = m_use;
+      if (j > 0 && rescale) {
+        // O may only be touched once the previous PV MMA has finished
+        ok = wait_bar(&sm.o_bar, (j - 1) & 1, v.err, dead);
+        if (ok) {
+          tc::fence_after_sync();
+          const uint32_t t_o = tbase + lane_off + kColO;
+#pragma unroll
+          for (int c4 = 0; c4 < kD / 32; ++c4) {
+            float o[32];
+            tc::ld32(t_o + 32 * c4, reinterpret_cast<uint32_t *>(o));
+            tc::wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= alpha;
+            tc::st32(t_o + 32 * c4, reinterpret_cast<const uint32_t *>(o));
+          }
+        }
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[buf]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && wait_bar(&sm.o_final, 0, v.err, dead)) {
+      tc::fence_after_sync();
+      const int qi = qt * kTile + r;
+      const float inv = 1.f / l_run;
+      const uint32_t t_o = tbase + lane_off + kColO;
+      __nv_bfloat16 *dst = a.out + ((int64_t)(tok0 + qi) * v.H + h) * kD;
+#pragma unroll
+      for (int c4 = 0; c4 < kD / 32; ++c4) {
+        float o[32];
+        tc::ld32(t_o + 32 * c4, reinterpret_cast<uint32_t *>(o));
+        tc::wait_ld();
+        if (qi < P) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pk[c] = tc::pack_bf16x2(o[2 * c] * inv, o[2 * c + 1] * inv);
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c4);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == kMmaWarp) tc::tmem_dealloc(tbase, kTmemCols);
+}
+
+// ------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// [tokens][H * 128] bf16 activations, 64 x 128 boxes, 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, const void *base, int64_t tokens, int H) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)H * kD, (cuuint64_t)tokens};
+  const cuuint64_t strides[1] = {(cuuint64_t)H * kD * 2};
+  const cuuint32_t box[2] = {64, kTile};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
+                              void *out, const int2 *tiles, cudaStream_t s) {
+  if (v.total_tiles == 0) return cudaSuccess;
+  if (v.D != kD || v.dtype != RSWA_BF16) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, v.total_tokens, v.H) || !make_tmap(&tk, k, v.total_tokens, v.H) ||
+      !make_tmap(&tv, vv, v.total_tokens, v.H))
+    return cudaErrorInvalidValue;
+  const int smem = (int)sizeof(PrefillSmem) + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  PrefillTcArgs args{v, tiles, (__nv_bfloat16 *)out};
+  prefill_tc_kernel<<<v.total_tiles * v.H, kThreads, smem, s>>>(tq, tk, tv, args);
+  return cudaGetLastError();
+}
+
+}  // namespace rswa

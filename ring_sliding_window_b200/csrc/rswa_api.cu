@@ -103,7 +103,7 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, i
   return p;
 }
 
-WsLayout layout_ws(const rswa_config *c, const DecodePlan &p) {
+WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &p) {
   const size_t B = (size_t)c->batch;
   WsLayout w;
   size_t off = 0;
@@ -114,9 +114,13 @@ WsLayout layout_ws(const rswa_config *c, const DecodePlan &p) {
   w.tok_base = off;    off = align256(off + (B + 1) * sizeof(int64_t));
   w.tile_base = off;   off = align256(off + (B + 1) * sizeof(int32_t));
   w.tile64_base = off; off = align256(off + (B + 1) * sizeof(int32_t));
+  size_t tiles = 0;
+  for (int b = 0; b < c->batch; ++b) tiles += (size_t)((plen[b] + kPrefillTile - 1) / kPrefillTile);
+  w.pf_tiles = off;    off = align256(off + tiles * sizeof(int2));
   w.pieces = off;      off = align256(off + (size_t)p.n_pieces * sizeof(DecodePiece));
   w.cta_piece = off;   off = align256(off + ((size_t)p.grid + 1) * sizeof(int32_t));
   w.bh_piece = off;    off = align256(off + (B * c->num_heads + 1) * sizeof(int32_t));
+  w.bh_count = off;    off = align256(off + (B * c->num_heads) * sizeof(int32_t));
   w.part_ml = off;     off = align256(off + (size_t)p.n_pieces * sizeof(float2));
   w.part_o = off;      off = align256(off + (size_t)p.n_pieces * c->head_dim * sizeof(float));
   w.total = off;
@@ -149,7 +153,7 @@ size_t rswa_workspace_bytes(const rswa_config *cfg, const int64_t *prefill_len) 
   if (dev < 0) return 0;
   const DecodePlan p =
       plan_decode(cfg, prefill_len, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
-  return layout_ws(cfg, p).total;
+  return layout_ws(cfg, prefill_len, p).total;
 }
 
 rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len,
@@ -182,7 +186,7 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   s->device = dev;
   s->num_sms = sm_count(dev);
   s->plan = plan_decode(cfg, prefill_len, s->num_sms, decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
-  s->ws = layout_ws(cfg, s->plan);
+  s->ws = layout_ws(cfg, prefill_len, s->plan);
   if (workspace_size < s->ws.total) {
     delete s;
     return RSWA_ENOMEM;
@@ -208,6 +212,15 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
     tl[b + 1] = tl[b] + (int32_t)((prefill_len[b] + kPrefillTile - 1) / kPrefillTile);
     tl64[b + 1] = tl64[b] + (int32_t)((prefill_len[b] + kSimtTile - 1) / kSimtTile);
     max_plen = std::max(max_plen, (int)prefill_len[b]);
+  }
+  {
+    // prefill query tiles, longest causal row range first
+    std::vector<int2> tiles;
+    for (int b = 0; b < B; ++b)
+      for (int qt = 0; qt * kPrefillTile < prefill_len[b]; ++qt) tiles.push_back(make_int2(b, qt));
+    std::stable_sort(tiles.begin(), tiles.end(),
+                     [](const int2 &x, const int2 &y) { return x.y > y.y; });
+    memcpy(at(s->ws.pf_tiles), tiles.data(), tiles.size() * sizeof(int2));
   }
   memcpy(at(s->ws.pieces), s->plan.pieces.data(), s->plan.pieces.size() * sizeof(DecodePiece));
   memcpy(at(s->ws.cta_piece), s->plan.cta_piece.data(), s->plan.cta_piece.size() * sizeof(int32_t));
@@ -237,9 +250,11 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   v.tok_base = (const int64_t *)(w + s->ws.tok_base);
   v.tile_base = (const int32_t *)(w + s->ws.tile_base);
   v.tile64_base = (const int32_t *)(w + s->ws.tile64_base);
+  v.pf_tiles = (const int2 *)(w + s->ws.pf_tiles);
   v.pieces = (const DecodePiece *)(w + s->ws.pieces);
   v.cta_piece = (const int32_t *)(w + s->ws.cta_piece);
   v.bh_piece = (const int32_t *)(w + s->ws.bh_piece);
+  v.bh_count = (int *)(w + s->ws.bh_count);
   v.part_ml = (float2 *)(w + s->ws.part_ml);
   v.part_o = (float *)(w + s->ws.part_o);
   v.decode_grid = s->plan.grid;
@@ -279,7 +294,10 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = launch_cache_fill(s->dv, k, v, s->k_cache[(size_t)layer], s->v_cache[(size_t)layer], st);
   if (e == cudaSuccess) {
-    e = launch_prefill_simt(s->dv, q, k, v, out, st);
+    if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128)
+      e = launch_prefill_tc(s->dv, q, k, v, out, s->dv.pf_tiles, st);
+    else
+      e = launch_prefill_simt(s->dv, q, k, v, out, st);
   }
   if (e != cudaSuccess) return RSWA_ECUDA;
   s->layer_ready[(size_t)layer] = 1;
@@ -295,7 +313,7 @@ rswa_status rswa_decode_step(rswa_state *s, int32_t layer, const void *q, const 
   if (!s->layer_ready[(size_t)layer]) return RSWA_ESTATE;
   if (current_device() != s->device) return RSWA_EINVAL;
   return from_cuda(launch_decode(s->dv, q, k_new, v_new, s->k_cache[(size_t)layer],
-                                 s->v_cache[(size_t)layer], out, (cudaStream_t)stream));
+                                 s->v_cache[(size_t)layer], out, (cudaStream_t)stream, true));
 }
 
 rswa_status rswa_advance(rswa_state *s, void *stream) {
