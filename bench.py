@@ -468,7 +468,7 @@ def run_also(w, args, flush, s, hbm_peak, tc_peak):
     rig.st.close()
     del rig
     torch.cuda.empty_cache()
-    if w.name == "multi_page_decode" and not args.skip_prefill_also:
+    if w.name in ("multi_page_decode", "near_max_context") and not args.skip_prefill_also:
         w1 = synth.Workload(w.name, w.cfg_id, w.dtype, w.batch, 2, w.heads, w.head_dim, w.window,
                             w.prefill_lens, 0)
         rig = DecodeRig(w1, 0, "prefill", s)
