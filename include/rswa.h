@@ -197,6 +197,10 @@ rswa_status rswa_check_device_error(rswa_state *state, void *stream);
 /* Static description of a status code. */
 const char *rswa_status_string(rswa_status status);
 
+/* Description of the CUDA error behind the calling thread's most recent
+ * RSWA_ECUDA ("no error" if there was none).  Static storage. */
+const char *rswa_last_cuda_error(void);
+
 /* ---- Allocation-free decode step --------------------------------------
  * This call has no counterpart in the paper; it exists for callers that
  * cannot hand the library a workspace.  A plugin hosted by another runtime

@@ -30,7 +30,7 @@ struct WsLayout {
   size_t tok_base;   // int64 [B+1] sum_{b'<b} P_b'
   size_t tile_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kPrefillTile)
   size_t tile64_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kSimtTile)
-  size_t pf_tiles;   // int2 [total_tiles] (b, query tile), longest first
+  size_t pf_blocks;  // int4 [n_pf_blocks] (b, h, first query tile, tiles 1|2)
   size_t pieces;     // DecodePiece [n_pieces]
   size_t cta_piece;  // int32 [G+1] first piece of each decode CTA
   size_t bh_piece;   // int32 [B*H+1] first piece of each (b, h)
@@ -64,7 +64,8 @@ struct DeviceView {
   const int64_t *tok_base;
   const int32_t *tile_base;
   const int32_t *tile64_base;
-  const int2 *pf_tiles;
+  const int4 *pf_blocks;
+  int n_pf_blocks;
   const DecodePiece *pieces;
   const int32_t *cta_piece;
   const int32_t *bh_piece;
@@ -109,7 +110,11 @@ cudaError_t launch_cache_fill(const DeviceView &v, const void *k, const void *vv
 cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,
                                 const void *vv, void *out, cudaStream_t s);
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, const int2 *tiles, cudaStream_t s);
+                              void *out, const int4 *blocks, int n_blocks, cudaStream_t s);
+
+// Prefill work list of the tensor-core kernel: blocks of two consecutive
+// 128-row query tiles of one (b, h), in launch order.
+std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms);
 cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
                          const int32_t *hist_len, int rows, int vocab, int n, int window,
                          int *err, cudaStream_t s);

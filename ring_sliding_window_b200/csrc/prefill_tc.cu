@@ -6,24 +6,28 @@
 // transformers path materialises the whole score matrix; here it is a
 // flash-style kernel that never leaves the chip with it.
 //
-// One CTA computes one 128-row query tile of one (sequence, head):
-//   warp 4      TMA producer: the Q tile once, then K and V tiles (128 keys x
+// One CTA computes two consecutive 128-row query tiles A = 2i and B = 2i + 1
+// of one (sequence, head); both read every K/V tile they need once from
+// shared memory:
+//   warp 8      TMA producer: Q_A and Q_B once, then K and V tiles (128 keys x
 //               128 dims, bf16, 128-byte swizzle) into a 2-stage ring;
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into a TMEM buffer
-//               (two buffers, 128 fp32 columns each), then O += P_j V_j with
-//               P_j read from TMEM (it overwrites S_j's columns as bf16 pairs);
-//               also owns the TMEM allocation;
-//   warps 0-3   softmax: thread r owns query row r (TMEM lane r).  It loads its
-//               S row, masks the diagonal tile, runs the online softmax in the
-//               log2 domain and writes P back to TMEM.  O (TMEM, fp32) is only
-//               rescaled when a warp's running max grows by more than 2^8;
-//               otherwise the stale max keeps every p <= 256, exact in the end
-//               because l uses the same max.  The epilogue divides by l and
-//               stores bf16 rows.
-// Query tiles are ordered longest-first (causal work grows with the tile
-// index).  Every mbarrier wait is bounded; on a timeout the kernel records it,
-// stops issuing work, waits (bounded) for what is in flight, frees TMEM and
-// returns.
+//   warp 9      MMA issuer (one thread) and TMEM owner (512 columns:
+//               S_A, S_B, O_A, O_B, 128 fp32 columns each).  Order per key
+//               tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so each softmax
+//               warpgroup works while the tensor core runs the other tile's
+//               MMAs.  P_X(j) overwrites S_X(j)'s columns as bf16 pairs and is
+//               the A operand (from TMEM) of PV_X(j);
+//   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: thread r of a
+//               warpgroup owns query row r (TMEM lane r).  It loads its S row,
+//               masks the diagonal tile, runs the online softmax in the log2
+//               domain and writes P back to TMEM.  O is only rescaled when a
+//               warp's running max grows by more than 2^8; otherwise the stale
+//               max keeps every p <= 256, exact in the end because l uses the
+//               same max.  The epilogue divides by l and stores bf16 rows.
+// Blocks are grouped by (sequence, head), longest first inside a group, so
+// the CTAs running together share their K/V tiles through L2.  Every mbarrier
+// wait is bounded; on a timeout the kernel records it, stops issuing work,
+// waits (bounded) for what is in flight, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,34 +45,35 @@ constexpr int kD = 128;      // head dim
 constexpr int kStages = 2;   // K/V ring depth
 constexpr int kHalfBytes = kTile * 64 * 2;   // one 64-column swizzled half: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;  // O accumulator
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 
+__host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)x * kTile; }        // 0, 128
+__host__ __device__ constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * kTile; } // 256, 384
+
 struct __align__(1024) PrefillSmem {
-  uint8_t q[kTileBytes];
+  uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   uint64_t q_full;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_bar;      // one phase per finished PV MMA
-  uint64_t o_final;    // the last PV MMA finished
-  uint64_t mma_done;   // everything the MMA thread issued finished
+  uint64_t s_full[2];    // per query tile: S_X(j) finished
+  uint64_t p_full[2];    // per query tile: P_X(j) written (4 warp arrivals)
+  uint64_t o_bar[2];     // per query tile: one phase per finished PV_X
+  uint64_t o_final[2];   // per query tile: the last PV_X finished
+  uint64_t mma_done;     // everything the MMA thread issued finished
   uint32_t tmem_base;
   int dead;
 };
 
 struct PrefillTcArgs {
   DeviceView v;
-  const int2 *tiles;  // (b, q_tile) longest-first
+  const int4 *blocks;  // (b, h, first query tile, number of tiles 1|2)
   __nv_bfloat16 *out;
 };
 
@@ -78,6 +83,28 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *er
   if (mbar_wait_bounded(bar, parity, err, RSWA_DEVERR_TIMEOUT)) return true;
   *dead = 1;
   return false;
+}
+
+// Issue the 8 K-steps of S = Q K^T (M = N = 128, K = 128 dims).
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTile, kTile, false, false);
+#pragma unroll
+  for (int kk = 0; kk < kD / 16; ++kk) {
+    const uint32_t off = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
+    tc::mma_ss(d_tmem, tc::sw128_desc(q_addr + off, 16, 1024),
+               tc::sw128_desc(k_addr + off, 16, 1024), idesc, kk > 0);
+  }
+}
+
+// Issue the 8 K-steps of O (+)= P V (M = 128 rows, N = 128 dims, K = 128 keys).
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr,
+                                         bool accumulate) {
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTile, kD, false, true);
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    tc::mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8,
+               tc::sw128_desc(v_addr + (uint32_t)kk * 2048, kHalfBytes, 1024), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -92,13 +119,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int tile_id = blockIdx.x / v.H;
-  const int h = blockIdx.x % v.H;
-  const int2 bt = a.tiles[tile_id];
-  const int b = bt.x, qt = bt.y;
+  const int4 blk = a.blocks[blockIdx.x];
+  const int b = blk.x, h = blk.y, qt0 = blk.z, ntiles = blk.w;
   const int P = v.plen[b];
   const int tok0 = (int)v.tok_base[b];
-  const int n_kv = qt + 1;  // causal: key tiles 0..qt
+  // key tiles needed by each query tile (causal): 0 .. qt
+  const int n_kv_a = qt0 + 1, n_kv_b = ntiles > 1 ? qt0 + 2 : 0;
+  const int n_kv_all = qt0 + ntiles;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
@@ -108,12 +135,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], 4);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], 4);
+      mbar_init(&sm.o_bar[x], 1);
+      mbar_init(&sm.o_final[x], 1);
     }
-    mbar_init(&sm.o_bar, 1);
-    mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
     sm.dead = 0;
     fence_mbar_init();
@@ -135,11 +162,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
       const int xh = h * kD;
-      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-      tc::tma_load_2d(sm.q, &tm_q, xh, tok0 + qt * kTile, &sm.q_full);
-      tc::tma_load_2d(sm.q + kHalfBytes, &tm_q, xh + 64, tok0 + qt * kTile, &sm.q_full);
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(ntiles * kTileBytes));
+      for (int x = 0; x < ntiles; ++x) {
+        const int y = tok0 + (qt0 + x) * kTile;
+        tc::tma_load_2d(sm.q[x], &tm_q, xh, y, &sm.q_full);
+        tc::tma_load_2d(sm.q[x] + kHalfBytes, &tm_q, xh + 64, y, &sm.q_full);
+      }
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < n_kv_all; ++j) {
         const int s = j % kStages;
         const uint32_t par = ((j / kStages) & 1) ^ 1;
         const int y = tok0 + j * kTile;
@@ -147,85 +177,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
         tc::tma_load_2d(sm.k[s], &tm_k, xh, y, &sm.k_full[s]);
         tc::tma_load_2d(sm.k[s] + kHalfBytes, &tm_k, xh + 64, y, &sm.k_full[s]);
-        if (!wait_bar(&sm.v_empty[s], par, v.err, dead)) {
-          issued = j + 1;  // K of tile j is in flight
-          break;
-        }
+        issued_k = j + 1;
+        if (!wait_bar(&sm.v_empty[s], par, v.err, dead)) break;
         mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
         tc::tma_load_2d(sm.v[s], &tm_v, xh, y, &sm.v_full[s]);
         tc::tma_load_2d(sm.v[s] + kHalfBytes, &tm_v, xh + 64, y, &sm.v_full[s]);
-        issued = j + 1;
+        issued_v = j + 1;
       }
       // every load issued has landed before the CTA may exit (bounded)
       mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / kStages) * kStages;  // last tile using stage s
-        const uint32_t par = (last / kStages) & 1;
-        mbar_wait_bounded(&sm.k_full[s], par, v.err, RSWA_DEVERR_TIMEOUT);
-        mbar_wait_bounded(&sm.v_full[s], par, v.err, RSWA_DEVERR_TIMEOUT);
+      for (int s = 0; s < kStages; ++s) {
+        if (s < issued_k) {
+          const int last = s + ((issued_k - 1 - s) / kStages) * kStages;
+          mbar_wait_bounded(&sm.k_full[s], (last / kStages) & 1, v.err, RSWA_DEVERR_TIMEOUT);
+        }
+        if (s < issued_v) {
+          const int last = s + ((issued_v - 1 - s) / kStages) * kStages;
+          mbar_wait_bounded(&sm.v_full[s], (last / kStages) & 1, v.err, RSWA_DEVERR_TIMEOUT);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(kTile, kTile, false, false);
-      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(kTile, kD, false, true);
-      const uint32_t q_addr = smem_u32(sm.q);
-      if (wait_bar(&sm.q_full, 0, v.err, dead)) {
-        for (int j = 0; j <= n_kv; ++j) {
-          if (j < n_kv) {
-            // S_j = Q K_j^T
-            const int s = j % kStages;
-            if (!wait_bar(&sm.k_full[s], (j / kStages) & 1, v.err, dead)) break;
-            tc::fence_after_sync();
-            const uint32_t k_addr = smem_u32(sm.k[s]);
-            const uint32_t d_s = tbase + kColS + (uint32_t)(j & 1) * kTile;
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32;
-              tc::mma_ss(d_s, tc::sw128_desc(q_addr + off, 16, 1024),
-                         tc::sw128_desc(k_addr + off, 16, 1024), idesc_qk, kk > 0);
+      const uint32_t q_addr0 = smem_u32(sm.q[0]);
+      bool ok = wait_bar(&sm.q_full, 0, v.err, dead) &&
+                wait_bar(&sm.k_full[0], 0, v.err, dead);
+      if (ok) {
+        tc::fence_after_sync();
+        for (int x = 0; x < ntiles; ++x) {
+          issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[0]));
+          tc::commit(&sm.s_full[x]);
+        }
+        tc::commit(&sm.k_empty[0]);
+      }
+      for (int j = 0; ok && j < n_kv_all; ++j) {
+        const int s = j % kStages;
+        const int s1 = (j + 1) % kStages;
+        bool k1_ready = false;  // K_{j+1} waited for
+        if (!(ok = wait_bar(&sm.v_full[s], (j / kStages) & 1, v.err, dead))) break;
+        for (int x = 0; x < ntiles; ++x) {
+          const int nkv = x == 0 ? n_kv_a : n_kv_b;
+          if (j >= nkv) continue;
+          // O_X += P_X(j) V_j
+          if (!(ok = wait_bar(&sm.p_full[x], j & 1, v.err, dead))) break;
+          tc::fence_after_sync();
+          issue_pv(tbase + col_o(x), tbase + col_s(x), smem_u32(sm.v[s]), j > 0);
+          tc::commit(&sm.o_bar[x]);
+          if (j == nkv - 1) tc::commit(&sm.o_final[x]);
+          // S_X(j+1) = Q_X K_{j+1}^T  (overwrites P_X(j): issued after PV_X(j))
+          if (j + 1 < nkv) {
+            if (!k1_ready) {
+              if (!(ok = wait_bar(&sm.k_full[s1], ((j + 1) / kStages) & 1, v.err, dead))) break;
+              tc::fence_after_sync();
+              k1_ready = true;
             }
-            tc::commit(&sm.s_full[j & 1]);
-            tc::commit(&sm.k_empty[s]);
-          }
-          if (j >= 1) {
-            // O += P_{j-1} V_{j-1}
-            const int jp = j - 1;
-            const int s = jp % kStages;
-            if (!wait_bar(&sm.p_full[jp & 1], (jp >> 1) & 1, v.err, dead)) break;
-            if (!wait_bar(&sm.v_full[s], (jp / kStages) & 1, v.err, dead)) break;
-            tc::fence_after_sync();
-            const uint32_t v_addr = smem_u32(sm.v[s]);
-            const uint32_t p_tmem = tbase + kColS + (uint32_t)(jp & 1) * kTile;
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              tc::mma_ts(tbase + kColO, p_tmem + (uint32_t)kk * 8,
-                         tc::sw128_desc(v_addr + (uint32_t)kk * 2048, kHalfBytes, 1024), idesc_pv,
-                         (jp > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc::commit(&sm.o_bar);
-            tc::commit(&sm.v_empty[s]);
-            if (jp == n_kv - 1) tc::commit(&sm.o_final);
+            issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[s1]));
+            tc::commit(&sm.s_full[x]);
           }
         }
+        if (!ok) break;
+        tc::commit(&sm.v_empty[s]);
+        if (k1_ready) tc::commit(&sm.k_empty[s1]);
       }
       tc::commit(&sm.mma_done);
       mbar_wait_bounded(&sm.mma_done, 0, v.err, RSWA_DEVERR_TIMEOUT);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = warp * 32 + lane;  // query row inside the tile = TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int x = warp >> 2;          // query tile of this warpgroup (0 = A, 1 = B)
+    const int wq = warp & 3;          // warp inside the warpgroup = TMEM lane quarter
+    const int r = wq * 32 + lane;     // query row inside the tile
+    const int qt = qt0 + x;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t t_s = tbase + lane_off + col_s(x);
+    const uint32_t t_o = tbase + lane_off + col_o(x);
     const float sl2 = v.scale * kLog2e;
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int buf = j & 1;
-      ok = wait_bar(&sm.s_full[buf], (j >> 1) & 1, v.err, dead);
+    const int nkv = x == 0 ? n_kv_a : n_kv_b;
+    bool ok = x < ntiles;
+    for (int j = 0; ok && j < nkv; ++j) {
+      ok = wait_bar(&sm.s_full[x], j & 1, v.err, dead);
       if (!ok) break;
       tc::fence_after_sync();
-      const uint32_t t_s = tbase + lane_off + kColS + (uint32_t)buf * kTile;
       float s[kTile];
       tc::ld32(t_s + 0, reinterpret_cast<uint32_t *>(s));
       tc::ld32(t_s + 32, reinterpret_cast<uint32_t *>(s) + 32);
@@ -267,11 +301,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_run = l_run * alpha + rs;
       m_run = m_use;
       if (j > 0 && rescale) {
-        // O may only be touched once the previous PV MMA has finished
-        ok = wait_bar(&sm.o_bar, (j - 1) & 1, v.err, dead);
+        // O_X may only be touched once PV_X(j-1) has finished (S_X(j) was
+        // issued after it, so this wait normally returns at once)
+        ok = wait_bar(&sm.o_bar[x], (j - 1) & 1, v.err, dead);
         if (ok) {
           tc::fence_after_sync();
-          const uint32_t t_o = tbase + lane_off + kColO;
 #pragma unroll
           for (int c4 = 0; c4 < kD / 32; ++c4) {
             float o[32];
@@ -286,14 +320,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[buf]);
+      if (lane == 0) mbar_arrive(&sm.p_full[x]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && wait_bar(&sm.o_final, 0, v.err, dead)) {
+    if (ok && x < ntiles && wait_bar(&sm.o_final[x], 0, v.err, dead)) {
       tc::fence_after_sync();
       const int qi = qt * kTile + r;
       const float inv = 1.f / l_run;
-      const uint32_t t_o = tbase + lane_off + kColO;
       __nv_bfloat16 *dst = a.out + ((int64_t)(tok0 + qi) * v.H + h) * kD;
 #pragma unroll
       for (int c4 = 0; c4 < kD / 32; ++c4) {
@@ -306,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 16; ++c) pk[c] = tc::pack_bf16x2(o[2 * c] * inv, o[2 * c + 1] * inv);
           uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c4);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 4; ++c)
+            d4[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
       }
     }
@@ -353,8 +387,8 @@ bool make_tmap(CUtensorMap *m, const void *base, int64_t tokens, int H) {
 }  // namespace
 
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, const int2 *tiles, cudaStream_t s) {
-  if (v.total_tiles == 0) return cudaSuccess;
+                              void *out, const int4 *blocks, int n_blocks, cudaStream_t s) {
+  if (n_blocks == 0) return cudaSuccess;
   if (v.D != kD || v.dtype != RSWA_BF16) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, v.total_tokens, v.H) || !make_tmap(&tk, k, v.total_tokens, v.H) ||
@@ -364,8 +398,8 @@ cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k,
   cudaError_t e =
       cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  PrefillTcArgs args{v, tiles, (__nv_bfloat16 *)out};
-  prefill_tc_kernel<<<v.total_tiles * v.H, kThreads, smem, s>>>(tq, tk, tv, args);
+  PrefillTcArgs args{v, blocks, (__nv_bfloat16 *)out};
+  prefill_tc_kernel<<<n_blocks, kThreads, smem, s>>>(tq, tk, tv, args);
   return cudaGetLastError();
 }
 

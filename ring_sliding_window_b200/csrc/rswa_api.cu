@@ -103,6 +103,35 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, i
   return p;
 }
 
+// Blocks of two consecutive query tiles of one (b, h).  A block's causal work
+// grows with its tile index.  (b, h) rings are taken in super-groups of about
+// one wave of blocks; inside a super-group blocks run longest first.  The
+// CTAs running together then share a few rings' K/V through L2, and the
+// last wave is not left with one long block.
+std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms) {
+  const int B = c->batch, H = c->num_heads;
+  std::vector<int4> out;
+  std::vector<int4> group;
+  int64_t group_blocks = 0;
+  auto flush = [&]() {
+    std::stable_sort(group.begin(), group.end(),
+                     [](const int4 &x, const int4 &y) { return x.z > y.z; });
+    out.insert(out.end(), group.begin(), group.end());
+    group.clear();
+    group_blocks = 0;
+  };
+  for (int b = 0; b < B; ++b) {
+    const int tiles = (int)((plen[b] + kPrefillTile - 1) / kPrefillTile);
+    for (int h = 0; h < H; ++h) {
+      for (int t0 = 0; t0 < tiles; t0 += 2) group.push_back(make_int4(b, h, t0, tiles - t0 >= 2 ? 2 : 1));
+      group_blocks += (tiles + 1) / 2;
+      if (group_blocks >= num_sms) flush();
+    }
+  }
+  flush();
+  return out;
+}
+
 WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &p) {
   const size_t B = (size_t)c->batch;
   WsLayout w;
@@ -114,9 +143,10 @@ WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &
   w.tok_base = off;    off = align256(off + (B + 1) * sizeof(int64_t));
   w.tile_base = off;   off = align256(off + (B + 1) * sizeof(int32_t));
   w.tile64_base = off; off = align256(off + (B + 1) * sizeof(int32_t));
-  size_t tiles = 0;
-  for (int b = 0; b < c->batch; ++b) tiles += (size_t)((plen[b] + kPrefillTile - 1) / kPrefillTile);
-  w.pf_tiles = off;    off = align256(off + tiles * sizeof(int2));
+  size_t blocks = 0;
+  for (int b = 0; b < c->batch; ++b)
+    blocks += (size_t)c->num_heads * (size_t)((plen[b] + 2 * kPrefillTile - 1) / (2 * kPrefillTile));
+  w.pf_blocks = off;   off = align256(off + blocks * sizeof(int4));
   w.pieces = off;      off = align256(off + (size_t)p.n_pieces * sizeof(DecodePiece));
   w.cta_piece = off;   off = align256(off + ((size_t)p.grid + 1) * sizeof(int32_t));
   w.bh_piece = off;    off = align256(off + (B * c->num_heads + 1) * sizeof(int32_t));
@@ -133,7 +163,13 @@ namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-rswa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RSWA_OK : RSWA_ECUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+rswa_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return RSWA_OK;
+  g_last_cuda_error = e;
+  return RSWA_ECUDA;
+}
 
 }  // namespace
 
@@ -213,15 +249,8 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
     tl64[b + 1] = tl64[b] + (int32_t)((prefill_len[b] + kSimtTile - 1) / kSimtTile);
     max_plen = std::max(max_plen, (int)prefill_len[b]);
   }
-  {
-    // prefill query tiles, longest causal row range first
-    std::vector<int2> tiles;
-    for (int b = 0; b < B; ++b)
-      for (int qt = 0; qt * kPrefillTile < prefill_len[b]; ++qt) tiles.push_back(make_int2(b, qt));
-    std::stable_sort(tiles.begin(), tiles.end(),
-                     [](const int2 &x, const int2 &y) { return x.y > y.y; });
-    memcpy(at(s->ws.pf_tiles), tiles.data(), tiles.size() * sizeof(int2));
-  }
+  const std::vector<int4> pf_blocks = plan_prefill_blocks(cfg, prefill_len, s->num_sms);
+  memcpy(at(s->ws.pf_blocks), pf_blocks.data(), pf_blocks.size() * sizeof(int4));
   memcpy(at(s->ws.pieces), s->plan.pieces.data(), s->plan.pieces.size() * sizeof(DecodePiece));
   memcpy(at(s->ws.cta_piece), s->plan.cta_piece.data(), s->plan.cta_piece.size() * sizeof(int32_t));
   memcpy(at(s->ws.bh_piece), s->plan.bh_piece.data(), s->plan.bh_piece.size() * sizeof(int32_t));
@@ -231,7 +260,7 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) {
     delete s;
-    return RSWA_ECUDA;
+    return from_cuda(e);
   }
 
   uint8_t *w = (uint8_t *)workspace;
@@ -250,7 +279,8 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   v.tok_base = (const int64_t *)(w + s->ws.tok_base);
   v.tile_base = (const int32_t *)(w + s->ws.tile_base);
   v.tile64_base = (const int32_t *)(w + s->ws.tile64_base);
-  v.pf_tiles = (const int2 *)(w + s->ws.pf_tiles);
+  v.pf_blocks = (const int4 *)(w + s->ws.pf_blocks);
+  v.n_pf_blocks = (int)pf_blocks.size();
   v.pieces = (const DecodePiece *)(w + s->ws.pieces);
   v.cta_piece = (const int32_t *)(w + s->ws.cta_piece);
   v.bh_piece = (const int32_t *)(w + s->ws.bh_piece);
@@ -295,11 +325,11 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
   cudaError_t e = launch_cache_fill(s->dv, k, v, s->k_cache[(size_t)layer], s->v_cache[(size_t)layer], st);
   if (e == cudaSuccess) {
     if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128)
-      e = launch_prefill_tc(s->dv, q, k, v, out, s->dv.pf_tiles, st);
+      e = launch_prefill_tc(s->dv, q, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, st);
     else
       e = launch_prefill_simt(s->dv, q, k, v, out, st);
   }
-  if (e != cudaSuccess) return RSWA_ECUDA;
+  if (e != cudaSuccess) return from_cuda(e);
   s->layer_ready[(size_t)layer] = 1;
   return RSWA_OK;
 }
@@ -372,6 +402,10 @@ rswa_status rswa_check_device_error(rswa_state *s, void *stream) {
   if (word & RSWA_DEVERR_TIMEOUT) return RSWA_ETIMEOUT;
   if (word) return RSWA_EDEVICE;
   return RSWA_OK;
+}
+
+const char *rswa_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
 }
 
 const char *rswa_status_string(rswa_status st) {

@@ -28,7 +28,7 @@ EXPORTED = (
     "rswa_cache_bytes", "rswa_workspace_bytes", "rswa_state_create", "rswa_state_destroy",
     "rswa_cache_offset", "rswa_prefill", "rswa_decode_step", "rswa_advance", "rswa_reset_ring",
     "rswa_ngram_mask", "rswa_get_ring", "rswa_check_device_error", "rswa_status_string",
-    "rswa_decode_step_noalloc",
+    "rswa_decode_step_noalloc", "rswa_last_cuda_error",
 )
 RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -36,7 +36,10 @@ RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
 class RswaError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} ({status})")
+        msg = f"{what}: {status_string(status)} ({status})"
+        if status == RSWA_ECUDA:
+            msg += f": {lib.rswa_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 class rswa_config(ctypes.Structure):
@@ -75,6 +78,8 @@ lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
 lib.rswa_decode_step_noalloc.argtypes = [_cfgp, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.rswa_decode_step_noalloc.restype = ctypes.c_int
+lib.rswa_last_cuda_error.argtypes = []
+lib.rswa_last_cuda_error.restype = ctypes.c_char_p
 lib.rswa_status_string.argtypes = [ctypes.c_int]
 lib.rswa_status_string.restype = ctypes.c_char_p
 for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_decode_step",
