@@ -50,6 +50,12 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// 1 in kEmuEvery exponential pairs uses the FMA-pipe exp2 (0: none, every
+// exponential on MUFU).  Build-time knob: -DRSWA_EXP2_FMA_EVERY=N.
+#ifndef RSWA_EXP2_FMA_EVERY
+#define RSWA_EXP2_FMA_EVERY 0
+#endif
+constexpr int kEmuEvery = RSWA_EXP2_FMA_EVERY;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)x * kTile; }        // 0, 128
@@ -271,9 +277,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kTile; ++c)
           if (c > r) s[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max as an 8-way tree (a single running max would be a 128-deep
+      // dependency chain)
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, s[c]);
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= sl2;
       const float m_new = fmaxf(m_run, mx);
       const bool need = j > 0 && m_new > m_run + kRescaleThreshold;
@@ -285,19 +297,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_use = m_new;
         alpha = tc::ex2(m_run - m_new);
       }
-      float rs = 0.f;
+      float rs8[8];  // row sum as 8 partial sums
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = tc::ex2(fmaf(s[64 * half + 2 * c], sl2, -m_use));
-          const float p1 = tc::ex2(fmaf(s[64 * half + 2 * c + 1], sl2, -m_use));
-          rs += p0 + p1;
+          const float x0 = fmaf(s[64 * half + 2 * c], sl2, -m_use);
+          const float x1 = fmaf(s[64 * half + 2 * c + 1], sl2, -m_use);
+          // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
+          const bool emu = kEmuEvery > 0 && (c % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
+          const float p0 = emu ? tc::exp2_fma(x0) : tc::ex2(x0);
+          const float p1 = emu ? tc::exp2_fma(x1) : tc::ex2(x1);
+          rs8[c & 7] += p0 + p1;
           pk[c] = tc::pack_bf16x2(p0, p1);
         }
         tc::st32(t_s + 32 * half, pk);
       }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l_run = l_run * alpha + rs;
       m_run = m_use;
       if (j > 0 && rescale) {

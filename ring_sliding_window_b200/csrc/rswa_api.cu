@@ -110,6 +110,11 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, i
 // last wave is not left with one long block.
 std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms) {
   const int B = c->batch, H = c->num_heads;
+  // Pairs of tiles halve the K/V traffic per query row, but a batch too
+  // small to give every SM a pair runs faster with one tile per CTA.
+  int64_t pairs = 0;
+  for (int b = 0; b < B; ++b) pairs += (int64_t)H * ((plen[b] + 2 * kPrefillTile - 1) / (2 * kPrefillTile));
+  const int per_block = pairs >= num_sms ? 2 : 1;
   std::vector<int4> out;
   std::vector<int4> group;
   int64_t group_blocks = 0;
@@ -123,8 +128,9 @@ std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen,
   for (int b = 0; b < B; ++b) {
     const int tiles = (int)((plen[b] + kPrefillTile - 1) / kPrefillTile);
     for (int h = 0; h < H; ++h) {
-      for (int t0 = 0; t0 < tiles; t0 += 2) group.push_back(make_int4(b, h, t0, tiles - t0 >= 2 ? 2 : 1));
-      group_blocks += (tiles + 1) / 2;
+      for (int t0 = 0; t0 < tiles; t0 += per_block)
+        group.push_back(make_int4(b, h, t0, tiles - t0 >= per_block ? per_block : 1));
+      group_blocks += (tiles + per_block - 1) / per_block;
       if (group_blocks >= num_sms) flush();
     }
   }
@@ -143,9 +149,9 @@ WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &
   w.tok_base = off;    off = align256(off + (B + 1) * sizeof(int64_t));
   w.tile_base = off;   off = align256(off + (B + 1) * sizeof(int32_t));
   w.tile64_base = off; off = align256(off + (B + 1) * sizeof(int32_t));
-  size_t blocks = 0;
+  size_t blocks = 0;  // upper bound: one tile per block
   for (int b = 0; b < c->batch; ++b)
-    blocks += (size_t)c->num_heads * (size_t)((plen[b] + 2 * kPrefillTile - 1) / (2 * kPrefillTile));
+    blocks += (size_t)c->num_heads * (size_t)((plen[b] + kPrefillTile - 1) / kPrefillTile);
   w.pf_blocks = off;   off = align256(off + blocks * sizeof(int4));
   w.pieces = off;      off = align256(off + (size_t)p.n_pieces * sizeof(DecodePiece));
   w.cta_piece = off;   off = align256(off + ((size_t)p.grid + 1) * sizeof(int32_t));

@@ -145,6 +145,29 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, to take part of the softmax's exponentials off the
+// MUFU unit.  Range reduction x = j + f, j = rint(x) (read from the low
+// mantissa bits of x + 1.5 * 2^23), f in [-1/2, 1/2]; 2^f by the degree-3
+// minimax polynomial (relative error) whose float32 coefficients
+// gen_exp2_poly.py derives with the Remez exchange algorithm; 2^j is added to
+// the exponent field.  Max relative error 7.5e-5 for x in [-125, 126];
+// x below -125 (including -inf) is clamped there and returns 2^-125 instead
+// of 0, which no softmax row sum can see next to its maximum term.
+constexpr float kExp2C0 = 0x1.fff692p-1f;
+constexpr float kExp2C1 = 0x1.62f31ap-1f;
+constexpr float kExp2C2 = 0x1.f0de1ap-3f;
+constexpr float kExp2C3 = 0x1.c3f76p-5f;
+
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23
+  const float j = t - 12582912.0f;  // rint(x)
+  const float f = x - j;
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  const int ji = __float_as_int(t) - 0x4B400000;
+  return __int_as_float(__float_as_int(p) + (ji << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -18,7 +18,9 @@ from typing import Optional, Sequence
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG, "librswa.so")
+# RSWA_LIBRARY may point at another build of the same library (e.g. one built
+# with different compile-time tuning); the default is the in-tree build.
+_LIB_PATH = os.environ.get("RSWA_LIBRARY") or os.path.join(_PKG, "librswa.so")
 
 RSWA_OK, RSWA_EINVAL, RSWA_ENOMEM, RSWA_ECUDA, RSWA_ESTATE, RSWA_ETIMEOUT, RSWA_EDEVICE = range(7)
 RSWA_F32, RSWA_BF16 = 0, 1
