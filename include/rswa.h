@@ -148,9 +148,15 @@ rswa_status rswa_prefill(rswa_state *state, int32_t layer, const void *q, const 
  *                                    ring overwrite are the same formula;
  *   cache[slot] <- (k_new, v_new);
  *   out   = softmax attention of q over slots [0, P_b + min(t_b + 1, W)).
- * The write and the attention are one fused split-K kernel followed by a
- * combine kernel.  Safe to capture in a CUDA graph (no host-side state
- * changes per step).  RSWA_ESTATE if the layer was never prefilled. */
+ * The write, the attention and the split-K combine are one kernel.  Safe to
+ * capture in a CUDA graph (no host-side state changes per step).
+ * The kernel uses programmatic dependent launch: it may start while the
+ * previous kernel in the stream is still running if that kernel lets its
+ * dependents start early (griddepcontrol.launch_dependents), and it then
+ * reads prompt rows (slots < P_b) of this layer's cache before waiting for
+ * that kernel.  A kernel that writes prompt rows must therefore not release
+ * its dependents early; everything else is read after the wait.
+ * RSWA_ESTATE if the layer was never prefilled. */
 rswa_status rswa_decode_step(rswa_state *state, int32_t layer, const void *q, const void *k_new,
                              const void *v_new, void *out, void *stream);
 

@@ -79,10 +79,6 @@ struct DecodeArgs {
   void *out;
 };
 
-__device__ __forceinline__ int64_t seg_offset_rows(const DeviceView &v, int b, int h, int plen) {
-  // first row (slot 0) of ring (b, h) in units of rows
-  return (int64_t)v.H * v.slot_base[b] + (int64_t)h * (plen + v.W);
-}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
@@ -96,6 +92,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   const int lane = threadIdx.x & 31;
   const int p_begin = v.cta_piece[blockIdx.x];
   const int p_end = v.cta_piece[blockIdx.x + 1];
+  // the work plan is written once when the state is built, so this CTA's
+  // first piece can be fetched before the grid-dependency wait below
+  const DecodePiece first_piece = v.pieces[p_begin];
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -105,30 +104,54 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     fence_mbar_init();
   }
   __syncthreads();
-  // Everything above touched only this launch's shared memory and the work
-  // tables written when the state was built; from here on the kernel reads
-  // q/k_new/v_new, the ring counters and the cache, which earlier kernels in
-  // the stream may still be producing.
+
+  // Prompt rows (slots < P_b) are written only by the prefill's cache fill
+  // or by the caller, never by a kernel that lets its dependents start early
+  // (only this kernel and the ring advance do, and neither writes a prompt
+  // row).  So the first stages of this CTA's first piece that lie wholly in
+  // the prompt can be requested before the grid-dependency wait; this
+  // overlaps their memory latency with the tail of the previous layer.
+  int pre_stages = 0;
+  if (warp == S::kConsumerWarps && lane == 0) {
+    const DecodePiece &pc = first_piece;
+    const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
+    const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
+    for (int k0 = pc.key_begin; k0 < pc.key_end && pre_stages < S::kStages;
+         k0 += S::kStageRows) {
+      const int rows = (pc.key_end - k0) < S::kStageRows ? (pc.key_end - k0) : S::kStageRows;
+      if (k0 + rows > pc.plen) break;
+      const uint32_t bytes = (uint32_t)rows * S::kRowBytes;
+      mbar_arrive_expect_tx(&sm.full[pre_stages], 2 * bytes);
+      bulk_g2s(sm.k[pre_stages], kbase + (int64_t)k0 * S::kRowBytes, bytes, &sm.full[pre_stages]);
+      bulk_g2s(sm.v[pre_stages], vbase + (int64_t)k0 * S::kRowBytes, bytes, &sm.full[pre_stages]);
+      ++pre_stages;
+    }
+  }
+  // From here on the kernel reads q/k_new/v_new, the ring counters and ring
+  // rows of the cache, which earlier kernels in the stream may still be
+  // producing.
   grid_dependency_wait();
   allow_dependents();
 
   if (warp == S::kConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane != 0) return;
-    int stage = 0;
-    uint32_t round = 0;
+    int stage = pre_stages % S::kStages;
+    uint32_t round = pre_stages / S::kStages;
     bool dead = false;
     for (int p = p_begin; p < p_end && !dead; ++p) {
-      const DecodePiece pc = v.pieces[p];
-      const int b = pc.bh / v.H, h = pc.bh % v.H;
-      const int plen = v.plen[b];
-      const int64_t t = v.t[b];
-      const int valid = plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
-      const int ke = pc.key_end < valid ? pc.key_end : valid;
-      const int64_t row0 = seg_offset_rows(v, b, h, plen);
-      const uint8_t *kbase = (const uint8_t *)a.kc + row0 * S::kRowBytes;
-      const uint8_t *vbase = (const uint8_t *)a.vc + row0 * S::kRowBytes;
-      for (int k0 = pc.key_begin; k0 < ke; k0 += S::kStageRows) {
+      const DecodePiece pc = p == p_begin ? first_piece : v.pieces[p];
+      // a piece wholly inside the prompt needs no ring counter
+      int ke = pc.key_end;
+      if (ke > pc.plen) {
+        const int64_t t = v.t[pc.b];
+        const int valid = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
+        ke = ke < valid ? ke : valid;
+      }
+      const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
+      const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
+      const int k_first = pc.key_begin + (p == p_begin ? pre_stages * S::kStageRows : 0);
+      for (int k0 = k_first; k0 < ke; k0 += S::kStageRows) {
         const int rows = (ke - k0) < S::kStageRows ? (ke - k0) : S::kStageRows;
         if (!mbar_wait_bounded(&sm.empty[stage], (round & 1) ^ 1, v.err, RSWA_DEVERR_TIMEOUT)) {
           dead = true;
@@ -156,15 +179,17 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   bool dead = false;
 
   for (int p = p_begin; p < p_end; ++p) {
-    const DecodePiece pc = v.pieces[p];
-    const int b = pc.bh / v.H, h = pc.bh % v.H;
-    const int plen = v.plen[b];
-    const int64_t t = v.t[b];
-    const int valid = plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
-    const int wslot = plen + (int)(t % v.W);
-    const int ke = pc.key_end < valid ? pc.key_end : valid;
+    const DecodePiece pc = p == p_begin ? first_piece : v.pieces[p];
+    // ring position: only pieces reaching past the prompt need it
+    int ke = pc.key_end, wslot = -1;
+    if (ke > pc.plen) {
+      const int64_t t = v.t[pc.b];
+      const int valid = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
+      wslot = pc.plen + (int)(t % v.W);
+      ke = ke < valid ? ke : valid;
+    }
     const bool owner = wslot >= pc.key_begin && wslot < pc.key_end;
-    const int64_t in_off = ((int64_t)b * v.H + h) * D;  // element offset into [B][H][D]
+    const int64_t in_off = ((int64_t)pc.b * v.H + pc.h) * D;  // element offset into [B][H][D]
 
     // q slice of this lane, pre-scaled into the log2 domain
     float qf[S::kEPL];
@@ -184,7 +209,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
       // ring write of this step + shared-memory copy for the substitution
       const uint8_t *kn = (const uint8_t *)a.k_new + in_off * (int64_t)sizeof(T);
       const uint8_t *vn = (const uint8_t *)a.v_new + in_off * (int64_t)sizeof(T);
-      const int64_t wrow = seg_offset_rows(v, b, h, plen) + wslot;
+      const int64_t wrow = pc.row0 + wslot;
       uint8_t *kdst = (uint8_t *)a.kc + wrow * S::kRowBytes;
       uint8_t *vdst = (uint8_t *)a.vc + wrow * S::kRowBytes;
       for (int c = tid; c < 2 * S::kChunks; c += 128) {
@@ -296,21 +321,28 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         for (int gg = 0; gg < S::kGroups; ++gg) L = fmaf(sm.red_l[gg], exp2f(sm.red_m[gg] - M), L);
       v.part_ml[p] = make_float2(M, L);
     }
-    // -------- publish the partial; the last piece of this (b, h) merges
-    __threadfence();
+    // -------- publish the partial; the last piece of this (b, h) merges.
+    // The barrier orders every thread's partial stores before thread 0's
+    // acq_rel atomic, whose release makes them visible device-wide and whose
+    // acquire (in the last CTA) orders the merge's loads after all of them.
     named_bar_sync(1, 128);
-    const int p0 = v.bh_piece[pc.bh], np = v.bh_piece[pc.bh + 1] - p0;
+    const int p0 = pc.first, np = pc.count;
+    const int bh = pc.b * v.H + pc.h;
     if (tid == 0) {
       int last = 1;
       if (np > 1) {
-        last = atomicAdd(&v.bh_count[pc.bh], 1) == np - 1;
-        if (last) v.bh_count[pc.bh] = 0;  // re-arm for the next launch
+        int old;
+        asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;"
+                     : "=r"(old)
+                     : "l"(v.bh_count + bh)
+                     : "memory");
+        last = old == np - 1;
+        if (last) v.bh_count[bh] = 0;  // re-arm for the next launch
       }
       sm.is_last = last;
     }
     named_bar_sync(1, 128);
     if (sm.is_last) {
-      __threadfence();
       // Thread tid merges output element tid.  Partials are read straight
       // from L2, kMergeBatch at a time with every load of a batch in flight
       // together, merged online by log-sum-exp.
@@ -340,7 +372,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         }
         Mg = Mc;
       }
-      if (tid < D) ((T *)a.out)[(int64_t)pc.bh * D + tid] = from_float<T>(acc / Lg);
+      if (tid < D) ((T *)a.out)[(int64_t)bh * D + tid] = from_float<T>(acc / Lg);
     }
   }
 }

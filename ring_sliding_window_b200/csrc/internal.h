@@ -13,11 +13,17 @@ namespace rswa {
 
 // Split-K piece of the decode attention: keys [key_begin, key_end) of one
 // (b, h) ring, all processed by one CTA.  Pieces are listed in flattened
-// (b, h, key) order, so the pieces of one (b, h) are contiguous.
-struct DecodePiece {
-  int32_t bh;
-  int32_t key_begin;
-  int32_t key_end;
+// (b, h, key) order, so the pieces of one (b, h) are contiguous.  A piece
+// carries everything the kernel needs to start streaming, so one load of it
+// (made before the kernel's grid-dependency wait) replaces a chain of table
+// lookups.
+struct __align__(16) DecodePiece {
+  int64_t row0;       // cache row of slot 0 of ring (b, h), in rows of d elements
+  int32_t b, h;
+  int32_t key_begin, key_end;
+  int32_t plen;       // P_b
+  int32_t first;      // first piece of this (b, h)
+  int32_t count;      // pieces of this (b, h)
   int32_t cta;
 };
 

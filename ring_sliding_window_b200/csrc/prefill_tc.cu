@@ -56,6 +56,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define RSWA_EXP2_FMA_EVERY 0
 #endif
 constexpr int kEmuEvery = RSWA_EXP2_FMA_EVERY;
+// 1: the two softmax warpgroups take turns on their exponential loops
+// (A(0), B(0), A(1), B(1), ...), keeping them half a period apart so each
+// has the MUFU pipe to itself while the tensor core runs the other tile's
+// MMAs.  Build-time knob: -DRSWA_SOFTMAX_ALTERNATE=0|1.
+#ifndef RSWA_SOFTMAX_ALTERNATE
+#define RSWA_SOFTMAX_ALTERNATE 1
+#endif
+constexpr bool kAlternate = RSWA_SOFTMAX_ALTERNATE != 0;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)x * kTile; }        // 0, 128
@@ -73,6 +81,7 @@ struct __align__(1024) PrefillSmem {
   uint64_t o_bar[2];     // per query tile: one phase per finished PV_X
   uint64_t o_final[2];   // per query tile: the last PV_X finished
   uint64_t mma_done;     // everything the MMA thread issued finished
+  uint64_t exp_done[2];  // per query tile: its warpgroup finished tile j's exponentials
   uint32_t tmem_base;
   int dead;
 };
@@ -146,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[x], 4);
       mbar_init(&sm.o_bar[x], 1);
       mbar_init(&sm.o_final[x], 1);
+      mbar_init(&sm.exp_done[x], 4);
     }
     mbar_init(&sm.mma_done, 1);
     sm.dead = 0;
@@ -297,6 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_use = m_new;
         alpha = tc::ex2(m_run - m_new);
       }
+      // take turns with the other warpgroup: A(j) after B(j-1), B(j) after A(j)
+      if (kAlternate && ntiles > 1) {
+        if (x == 0 && j > 0) ok = wait_bar(&sm.exp_done[1], (j - 1) & 1, v.err, dead);
+        if (x == 1 && j < n_kv_a) ok = wait_bar(&sm.exp_done[0], j & 1, v.err, dead);
+        if (!ok) break;
+      }
       float rs8[8];  // row sum as 8 partial sums
 #pragma unroll
       for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
@@ -317,6 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::st32(t_s + 32 * half, pk);
       }
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      if (kAlternate && ntiles > 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.exp_done[x]);
+      }
       l_run = l_run * alpha + rs;
       m_run = m_use;
       if (j > 0 && rescale) {

@@ -84,9 +84,14 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, i
       while (seg_start[seg + 1] <= r0) ++seg;
       const int64_t e = std::min(r1, seg_start[seg + 1]);
       DecodePiece pc;
-      pc.bh = (int32_t)seg;
+      pc.b = (int32_t)(seg / (size_t)H);
+      pc.h = (int32_t)(seg % (size_t)H);
+      pc.row0 = seg_start[seg];  // rings are laid out back to back in (b, h) order
       pc.key_begin = (int32_t)(r0 - seg_start[seg]);
       pc.key_end = (int32_t)(e - seg_start[seg]);
+      pc.plen = (int32_t)plen[pc.b];
+      pc.first = 0;
+      pc.count = 0;
       pc.cta = (int32_t)cta;
       p.pieces.push_back(pc);
       r0 = e;
@@ -97,8 +102,13 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, i
   // first piece of each (b, h): pieces are in flattened order
   size_t i = 0;
   for (size_t bh = 0; bh <= (size_t)B * H; ++bh) {
-    while (i < p.pieces.size() && (size_t)p.pieces[i].bh < bh) ++i;
+    while (i < p.pieces.size() && (size_t)p.pieces[i].b * H + p.pieces[i].h < bh) ++i;
     p.bh_piece[bh] = (int32_t)i;
+  }
+  for (DecodePiece &pc : p.pieces) {
+    const size_t bh = (size_t)pc.b * H + pc.h;
+    pc.first = p.bh_piece[bh];
+    pc.count = p.bh_piece[bh + 1] - p.bh_piece[bh];
   }
   return p;
 }
