@@ -116,6 +116,49 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+DECODE_KERNEL_SOURCES = ("decode.cu", "ptx.cuh", "internal.h")
+
+
+def kernel_source_hash(files=DECODE_KERNEL_SOURCES) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "ring_sliding_window_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per decode-kernel launch from the committed ncu record, or
+    None when the kernel sources changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "decode_split_kernel_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_sha256") != kernel_source_hash() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def max_over_ranks(x: float) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return float(x)
+
+
+def aggregate_rate(steps_per_rank: int, max_total_ms: float, world: int) -> float:
+    """Whole-job rate: every rank ran `steps_per_rank` steps of its own replica
+    (weak scaling); the job took as long as its slowest rank."""
+    return world * steps_per_rank / (max_total_ms / 1e3)
+
+
 def kv_bytes_per_layer(w: synth.Workload, t_list):
     """Algorithmic bytes of one rswa_decode_step (one layer): K and V rows of
     every valid slot, q, k_new/v_new read, ring write, output write."""
@@ -371,13 +414,8 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(dev if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dev]))
     ms, ts, clocks = timed_tokens(rig, args.steps, args.warmup, flush, sampler)
-    total_ms = sum(ms)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    value = world * args.steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(ms))
+    value = aggregate_rate(args.steps, total_ms, world)
     kv_bytes = sum(w.layers * kv_bytes_per_layer(w, t) for t in ts)
     kv_gbs = kv_bytes / (sum(ms) / 1e3) / 1e9
 
@@ -389,13 +427,8 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- e2e through the public API with host buffers
     e2e_ms, h2d, d2h = e2e_tokens(rig, args.steps, args.warmup, flush)
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_total = float(tt.item())
-    e2e_value = world * args.steps / (e2e_total / 1e3)
+    e2e_total = max_over_ranks(sum(e2e_ms))
+    e2e_value = aggregate_rate(args.steps, e2e_total, world)
     pf_flops = prefill_flops_per_layer(w)
     pf_mean = statistics.mean(pf_ms) / 1e3
     assert rig.st.check() == 0, "device error word set during the run"
@@ -422,7 +455,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": achieved / hbm_peak, "peak_source": peak_src,
                      "frac_of_datasheet_8000": achieved / DATASHEET_HBM_GBS,
                      "algorithmic_bytes_per_launch": per_launch_bytes,
-                     "avg_launch_us": dur * 1e6, "traffic": None},
+                     "avg_launch_us": dur * 1e6, "traffic": measured_traffic(w.name)},
         "prefill": {"workload": w.name, "tflops": pf_flops / pf_mean / 1e12, "unit": "TFLOP/s",
                     "peak": tc_peak, "frac": pf_flops / pf_mean / 1e12 / tc_peak,
                     "frac_of_datasheet_2250": pf_flops / pf_mean / 1e12 / DATASHEET_BF16_TFLOPS,

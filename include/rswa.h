@@ -245,6 +245,16 @@ rswa_status rswa_decode_step_noalloc(const rswa_config *cfg, const int64_t *pref
                                      const void *q, const void *k_new, const void *v_new,
                                      void *out, int32_t *device_error, void *stream);
 
+/* ---- Fault injection (tests only) ---------------------------------------
+ * RSWA_FAULT_DROP_DECODE_COPIES: subsequent decode kernels of this state
+ * issue none of their cache copies, so every bounded wait in them runs out
+ * (about 1 s): the kernel records RSWA_DEVERR_TIMEOUT, finishes, and
+ * rswa_check_device_error returns RSWA_ETIMEOUT; outputs of those steps are
+ * garbage, the cache is untouched apart from the ring write.  flags = 0
+ * restores normal operation.  Enqueued on `stream` (pageable copy). */
+#define RSWA_FAULT_DROP_DECODE_COPIES 1
+rswa_status rswa_debug_inject_fault(rswa_state *state, int32_t flags, void *stream);
+
 /* Bits of a device error word. */
 #define RSWA_DEVERR_TIMEOUT 1
 #define RSWA_DEVERR_BAD_TOKEN 2

@@ -112,7 +112,12 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   // the prompt can be requested before the grid-dependency wait; this
   // overlaps their memory latency with the tail of the previous layer.
   int pre_stages = 0;
-  if (warp == S::kConsumerWarps && lane == 0) {
+  // Test-only fault injection: with RSWA_FAULT_DROP_DECODE_COPIES set the
+  // producer issues no copy at all, so every consumer wait runs out, records
+  // RSWA_DEVERR_TIMEOUT and the kernel still finishes.  The flag is written by
+  // a host copy, which a kernel launched after it never overlaps.
+  const bool drop_copies = (*v.fault & RSWA_FAULT_DROP_DECODE_COPIES) != 0;
+  if (warp == S::kConsumerWarps && lane == 0 && !drop_copies) {
     const DecodePiece &pc = first_piece;
     const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
     const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
@@ -135,7 +140,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
 
   if (warp == S::kConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (lane != 0) return;
+    if (lane != 0 || drop_copies) return;
     int stage = pre_stages % S::kStages;
     uint32_t round = pre_stages / S::kStages;
     bool dead = false;

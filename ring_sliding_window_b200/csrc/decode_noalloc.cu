@@ -114,6 +114,7 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
   v.dtype = cfg->dtype;
   v.scale = cfg->scale == 0.f ? 1.0f / sqrtf((float)cfg->head_dim) : cfg->scale;
   v.err = device_error ? (int *)device_error : (int *)(scratch + ws.err);
+  v.fault = (const int *)(scratch + ws.err) + 1;  // zero: the table image clears it
   v.t = (int64_t *)(scratch + ws.t);
   v.plen = (const int32_t *)(scratch + ws.plen);
   v.slot_base = (const int64_t *)(scratch + ws.slot_base);

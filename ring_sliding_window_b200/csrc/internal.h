@@ -64,6 +64,7 @@ struct DeviceView {
   int dtype;
   float scale;
   int *err;
+  const int *fault;  // fault-injection flags (tests only; 0 in normal use)
   int64_t *t;
   const int32_t *plen;
   const int64_t *slot_base;

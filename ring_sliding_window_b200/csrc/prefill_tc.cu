@@ -59,9 +59,10 @@ constexpr int kEmuEvery = RSWA_EXP2_FMA_EVERY;
 // 1: the two softmax warpgroups take turns on their exponential loops
 // (A(0), B(0), A(1), B(1), ...), keeping them half a period apart so each
 // has the MUFU pipe to itself while the tensor core runs the other tile's
-// MMAs.  Build-time knob: -DRSWA_SOFTMAX_ALTERNATE=0|1.
+// MMAs.  Build-time knob: -DRSWA_SOFTMAX_ALTERNATE=0|1; off by default
+// because on B200 it measured slightly slower (830 vs 845 TFLOP/s, multi-page).
 #ifndef RSWA_SOFTMAX_ALTERNATE
-#define RSWA_SOFTMAX_ALTERNATE 1
+#define RSWA_SOFTMAX_ALTERNATE 0
 #endif
 constexpr bool kAlternate = RSWA_SOFTMAX_ALTERNATE != 0;
 constexpr float kLog2e = 1.4426950408889634f;

@@ -289,6 +289,7 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   v.dtype = cfg->dtype;
   v.scale = s->cfg.scale;
   v.err = (int *)(w + s->ws.err);
+  v.fault = (const int *)(w + s->ws.err) + 1;
   v.t = (int64_t *)(w + s->ws.t);
   v.plen = (const int32_t *)(w + s->ws.plen);
   v.slot_base = (const int64_t *)(w + s->ws.slot_base);
@@ -418,6 +419,14 @@ rswa_status rswa_check_device_error(rswa_state *s, void *stream) {
   if (word & RSWA_DEVERR_TIMEOUT) return RSWA_ETIMEOUT;
   if (word) return RSWA_EDEVICE;
   return RSWA_OK;
+}
+
+rswa_status rswa_debug_inject_fault(rswa_state *s, int32_t flags, void *stream) {
+  if (!s || (flags & ~RSWA_FAULT_DROP_DECODE_COPIES) != 0) return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  // the host value is staged by the copy before the call returns
+  return from_cuda(cudaMemcpyAsync((int *)s->dv.fault, &flags, sizeof(int32_t),
+                                   cudaMemcpyHostToDevice, (cudaStream_t)stream));
 }
 
 const char *rswa_last_cuda_error(void) {

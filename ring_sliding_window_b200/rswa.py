@@ -30,8 +30,9 @@ EXPORTED = (
     "rswa_cache_bytes", "rswa_workspace_bytes", "rswa_state_create", "rswa_state_destroy",
     "rswa_cache_offset", "rswa_prefill", "rswa_decode_step", "rswa_advance", "rswa_reset_ring",
     "rswa_ngram_mask", "rswa_get_ring", "rswa_check_device_error", "rswa_status_string",
-    "rswa_decode_step_noalloc", "rswa_last_cuda_error",
+    "rswa_decode_step_noalloc", "rswa_last_cuda_error", "rswa_debug_inject_fault",
 )
+RSWA_FAULT_DROP_DECODE_COPIES = 1
 RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -80,6 +81,8 @@ lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
 lib.rswa_decode_step_noalloc.argtypes = [_cfgp, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.rswa_decode_step_noalloc.restype = ctypes.c_int
+lib.rswa_debug_inject_fault.argtypes = [_vp, ctypes.c_int32, _vp]
+lib.rswa_debug_inject_fault.restype = ctypes.c_int
 lib.rswa_last_cuda_error.argtypes = []
 lib.rswa_last_cuda_error.restype = ctypes.c_char_p
 lib.rswa_status_string.argtypes = [ctypes.c_int]
@@ -206,6 +209,12 @@ def rswa_decode_step_noalloc(cfg: rswa_config, prefill_len, n_generated, k_cache
                                         _ptr(k_cache), _ptr(v_cache), _ptr(q), _ptr(k_new),
                                         _ptr(v_new), _ptr(out), _ptr(device_error),
                                         _stream(stream)), "rswa_decode_step_noalloc")
+
+
+def rswa_debug_inject_fault(state, flags: int, stream=None) -> None:
+    """Test-only: make this state's decode kernels drop their copies (their
+    bounded waits then run out and report RSWA_ETIMEOUT); 0 restores."""
+    _check(lib.rswa_debug_inject_fault(state, int(flags), _stream(stream)), "rswa_debug_inject_fault")
 
 
 # ---------------------------------------------------------- owning helper

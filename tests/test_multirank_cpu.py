@@ -1,0 +1,69 @@
+"""The multi-GPU path of bench.py on CPU: replicas only (each rank runs its own
+copy of the workload, no data-path collective), timed as the max over ranks.
+Runs as two gloo ranks on 127.0.0.1."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, results):
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        per_rank_ms = [120.0, 150.0][rank]
+        mx = bench.max_over_ranks(per_rank_ms)
+        rate = bench.aggregate_rate(1000, mx, world)
+        results[rank] = (mx, rate)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_rate_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, results)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for r in range(2):
+        mx, rate = results[r]
+        assert mx == 150.0                       # every rank sees the slowest rank
+        assert rate == pytest.approx(2 * 1000 / 0.150)  # all ranks' steps / max time
+
+
+def test_single_process_aggregation():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.aggregate_rate(10, 1000.0, 1) == pytest.approx(10.0)
+
+
+def test_reference_arm_only_rank0_prints():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
