@@ -42,12 +42,15 @@ namespace {
 
 constexpr int kTile = 128;   // query rows and keys per tile
 constexpr int kD = 128;      // head dim
-constexpr int kStages = 2;   // K/V ring depth
+constexpr int kKStages = 2;  // K ring depth
+constexpr int kVStages = 3;  // V ring depth: a V tile is held until PV_B is done, and a
+                             // 32 KB tile load takes ~2.8 us under full load
 constexpr int kHalfBytes = kTile * 64 * 2;   // one 64-column swizzled half: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 8;   // Q and K loads
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10; // V loads
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // 1 in kEmuEvery exponential pairs uses the FMA-pipe exp2 (0: none, every
@@ -72,11 +75,11 @@ __host__ __device__ constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x 
 
 struct __align__(1024) PrefillSmem {
   uint8_t q[2][kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t k[kKStages][kTileBytes];
+  uint8_t v[kVStages][kTileBytes];
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2];    // per query tile: S_X(j) finished
   uint64_t p_full[2];    // per query tile: P_X(j) written (4 warp arrivals)
   uint64_t o_bar[2];     // per query tile: one phase per finished PV_X
@@ -145,9 +148,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
@@ -172,46 +177,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = sm.tmem_base;
   volatile int *dead = &sm.dead;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
+  if (warp == kProducerWarp || warp == kVProducerWarp) {
+    // ------------------------------------------------------------ producers
+    // warp 8 loads Q and the K ring, warp 10 the V ring, so a K load never
+    // waits behind a V slot that is still in use (and the other way round).
     if (lane == 0) {
-      tc::prefetch_tmap(&tm_q);
-      tc::prefetch_tmap(&tm_k);
-      tc::prefetch_tmap(&tm_v);
+      const bool is_k = warp == kProducerWarp;
       const int xh = h * kD;
-      mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(ntiles * kTileBytes));
-      for (int x = 0; x < ntiles; ++x) {
-        const int y = tok0 + (qt0 + x) * kTile;
-        tc::tma_load_2d(sm.q[x], &tm_q, xh, y, &sm.q_full);
-        tc::tma_load_2d(sm.q[x] + kHalfBytes, &tm_q, xh + 64, y, &sm.q_full);
+      const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+      const int nst = is_k ? kKStages : kVStages;
+      tc::prefetch_tmap(tm);
+      if (is_k) {
+        tc::prefetch_tmap(&tm_q);
+        mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(ntiles * kTileBytes));
+        for (int x = 0; x < ntiles; ++x) {
+          const int y = tok0 + (qt0 + x) * kTile;
+          tc::tma_load_2d(sm.q[x], &tm_q, xh, y, &sm.q_full);
+          tc::tma_load_2d(sm.q[x] + kHalfBytes, &tm_q, xh + 64, y, &sm.q_full);
+        }
       }
-      int issued_k = 0, issued_v = 0;
+      int issued = 0;
       for (int j = 0; j < n_kv_all; ++j) {
-        const int s = j % kStages;
-        const uint32_t par = ((j / kStages) & 1) ^ 1;
-        const int y = tok0 + j * kTile;
-        if (!wait_bar(&sm.k_empty[s], par, v.err, dead)) break;
-        mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
-        tc::tma_load_2d(sm.k[s], &tm_k, xh, y, &sm.k_full[s]);
-        tc::tma_load_2d(sm.k[s] + kHalfBytes, &tm_k, xh + 64, y, &sm.k_full[s]);
-        issued_k = j + 1;
-        if (!wait_bar(&sm.v_empty[s], par, v.err, dead)) break;
-        mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
-        tc::tma_load_2d(sm.v[s], &tm_v, xh, y, &sm.v_full[s]);
-        tc::tma_load_2d(sm.v[s] + kHalfBytes, &tm_v, xh + 64, y, &sm.v_full[s]);
-        issued_v = j + 1;
+        const int s = j % nst;
+        uint64_t *empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+        uint64_t *full = is_k ? &sm.k_full[s] : &sm.v_full[s];
+        uint8_t *dst = is_k ? sm.k[s] : sm.v[s];
+        if (!wait_bar(empty, ((j / nst) & 1) ^ 1, v.err, dead)) break;
+        mbar_arrive_expect_tx(full, kTileBytes);
+        tc::tma_load_2d(dst, tm, xh, tok0 + j * kTile, full);
+        tc::tma_load_2d(dst + kHalfBytes, tm, xh + 64, tok0 + j * kTile, full);
+        issued = j + 1;
       }
       // every load issued has landed before the CTA may exit (bounded)
-      mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
-      for (int s = 0; s < kStages; ++s) {
-        if (s < issued_k) {
-          const int last = s + ((issued_k - 1 - s) / kStages) * kStages;
-          mbar_wait_bounded(&sm.k_full[s], (last / kStages) & 1, v.err, RSWA_DEVERR_TIMEOUT);
-        }
-        if (s < issued_v) {
-          const int last = s + ((issued_v - 1 - s) / kStages) * kStages;
-          mbar_wait_bounded(&sm.v_full[s], (last / kStages) & 1, v.err, RSWA_DEVERR_TIMEOUT);
-        }
+      if (is_k) mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
+      for (int s = 0; s < nst && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / nst) * nst;
+        mbar_wait_bounded(is_k ? &sm.k_full[s] : &sm.v_full[s], (last / nst) & 1, v.err,
+                          RSWA_DEVERR_TIMEOUT);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -229,10 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::commit(&sm.k_empty[0]);
       }
       for (int j = 0; ok && j < n_kv_all; ++j) {
-        const int s = j % kStages;
-        const int s1 = (j + 1) % kStages;
+        const int s = j % kVStages;          // V stage of tile j
+        const int s1 = (j + 1) % kKStages;   // K stage of tile j + 1
         bool k1_ready = false;  // K_{j+1} waited for
-        if (!(ok = wait_bar(&sm.v_full[s], (j / kStages) & 1, v.err, dead))) break;
+        if (!(ok = wait_bar(&sm.v_full[s], (j / kVStages) & 1, v.err, dead))) break;
         for (int x = 0; x < ntiles; ++x) {
           const int nkv = x == 0 ? n_kv_a : n_kv_b;
           if (j >= nkv) continue;
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // S_X(j+1) = Q_X K_{j+1}^T  (overwrites P_X(j): issued after PV_X(j))
           if (j + 1 < nkv) {
             if (!k1_ready) {
-              if (!(ok = wait_bar(&sm.k_full[s1], ((j + 1) / kStages) & 1, v.err, dead))) break;
+              if (!(ok = wait_bar(&sm.k_full[s1], ((j + 1) / kKStages) & 1, v.err, dead))) break;
               tc::fence_after_sync();
               k1_ready = true;
             }
@@ -294,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int c = 8; c < kTile; c += 2) mx8[(c >> 1) & 7] = tc::fmax3(mx8[(c >> 1) & 7], s[c], s[c + 1]);
+      float mx = tc::fmax3(tc::fmax3(mx8[0], mx8[1], mx8[2]), tc::fmax3(mx8[3], mx8[4], mx8[5]),
+                           fmaxf(mx8[6], mx8[7]));
       mx *= sl2;
       const float m_new = fmaxf(m_run, mx);
       const bool need = j > 0 && m_new > m_run + kRescaleThreshold;
@@ -314,26 +316,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (x == 1 && j < n_kv_a) ok = wait_bar(&sm.exp_done[0], j & 1, v.err, dead);
         if (!ok) break;
       }
-      float rs8[8];  // row sum as 8 partial sums
+      uint64_t rs4[4];  // row sum as 4 packed pairs of partial sums
 #pragma unroll
-      for (int i = 0; i < 8; ++i) rs8[i] = 0.f;
+      for (int i = 0; i < 4; ++i) rs4[i] = 0;
+      const uint64_t sl2x2 = tc::f2_pack(sl2, sl2);
+      const uint64_t negm2 = tc::f2_pack(-m_use, -m_use);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float x0 = fmaf(s[64 * half + 2 * c], sl2, -m_use);
-          const float x1 = fmaf(s[64 * half + 2 * c + 1], sl2, -m_use);
+          // x = s * scale*log2(e) - m for the pair, one packed FMA
+          const uint64_t xx = tc::ffma2(tc::f2_pack(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]),
+                                        sl2x2, negm2);
+          const float x0 = tc::f2_lo(xx), x1 = tc::f2_hi(xx);
           // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
           const bool emu = kEmuEvery > 0 && (c % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
           const float p0 = emu ? tc::exp2_fma(x0) : tc::ex2(x0);
           const float p1 = emu ? tc::exp2_fma(x1) : tc::ex2(x1);
-          rs8[c & 7] += p0 + p1;
+          rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(p0, p1));
           pk[c] = tc::pack_bf16x2(p0, p1);
         }
         tc::st32(t_s + 32 * half, pk);
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      const uint64_t r01 = tc::fadd2(tc::fadd2(rs4[0], rs4[1]), tc::fadd2(rs4[2], rs4[3]));
+      const float rs = tc::f2_lo(r01) + tc::f2_hi(r01);
       if (kAlternate && ntiles > 1) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.exp_done[x]);
@@ -351,8 +358,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             float o[32];
             tc::ld32(t_o + 32 * c4, reinterpret_cast<uint32_t *>(o));
             tc::wait_ld();
+            const uint64_t a2 = tc::f2_pack(alpha, alpha);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] *= alpha;
+            for (int c = 0; c < 16; ++c) {
+              const uint64_t r = tc::fmul2(tc::f2_pack(o[2 * c], o[2 * c + 1]), a2);
+              o[2 * c] = tc::f2_lo(r);
+              o[2 * c + 1] = tc::f2_hi(r);
+            }
             tc::st32(t_o + 32 * c4, reinterpret_cast<const uint32_t *>(o));
           }
         }
