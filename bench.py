@@ -432,6 +432,7 @@ def run_ours(args, rank, world, local_rank):
     pf_flops = prefill_flops_per_layer(w)
     pf_mean = statistics.mean(pf_ms) / 1e3
     assert rig.st.check() == 0, "device error word set during the run"
+    dec_grid, dec_cluster = rig.st.decode_launch_shape()
     rig.st.close()
     del rig
     torch.cuda.empty_cache()
@@ -447,7 +448,10 @@ def run_ours(args, rank, world, local_rank):
                    "decode_from_t": 0, "step": "one token: all layers' rswa_decode_step + "
                    "rswa_advance + rswa_ngram_mask (n=35, window=128) as one CUDA graph",
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": f"replicas x{world}",
+                   "decode_launch": {"grid": dec_grid, "cluster_size": dec_cluster,
+                                     "split": "cluster per ring (DSMEM merge)" if dec_cluster
+                                     else "stream-K (workspace merge)"}},
         "kv_read_gbs": kv_gbs,
         "roofline": {"kernel": "decode_split_kernel (rswa_decode_step: ring write + split-K "
                                "attention + in-kernel combine)",

@@ -200,6 +200,20 @@ rswa_status rswa_get_ring(const rswa_state *state, int64_t *n_generated, int32_t
  * RSWA_OK, RSWA_ETIMEOUT or RSWA_EDEVICE.  Clears the word. */
 rswa_status rswa_check_device_error(rswa_state *state, void *stream);
 
+/* The launch shape rswa_decode_step uses for this state (host only, no
+ * synchronisation):
+ *  grid         : CTAs per decode launch;
+ *  cluster_size : 0 when the flattened key rows of all rings are split into
+ *                 `grid` equal ranges whose partials are merged through the
+ *                 workspace; C >= 2 when each (b, h) ring has a cluster of C
+ *                 CTAs that merge through distributed shared memory (chosen
+ *                 when all rings' clusters are resident at once).
+ * Either pointer may be NULL.  The environment variable RSWA_DECODE_SPLIT
+ * (`streamk` or `cluster`), read by rswa_state_create, overrides the choice
+ * where the cluster form fits. */
+rswa_status rswa_decode_launch_shape(const rswa_state *state, int32_t *grid,
+                                     int32_t *cluster_size);
+
 /* Static description of a status code. */
 const char *rswa_status_string(rswa_status status);
 

@@ -38,6 +38,7 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMergeBatch = 16;  // partials whose loads are in flight together in the merge
+constexpr int kMaxCluster = 16;  // CTAs per ring in the cluster variant
 
 template <typename T, int D>
 struct DecodeShape {
@@ -57,7 +58,7 @@ struct DecodeShape {
   static_assert(kEPL * 8 == D, "lane split must cover the row");
 };
 
-template <typename T, int D>
+template <typename T, int D, bool kCluster>
 struct __align__(128) DecodeSmem {
   using S = DecodeShape<T, D>;
   uint8_t k[S::kStages][S::kStageRows * S::kRowBytes];
@@ -68,6 +69,10 @@ struct __align__(128) DecodeSmem {
   float red_m[S::kGroups];
   float red_l[S::kGroups];
   int is_last;
+  // cluster variant: partials of the cluster's CTAs, written into the
+  // leader's copy through distributed shared memory
+  float cl_o[kCluster ? kMaxCluster : 1][D];
+  float2 cl_ml[kCluster ? kMaxCluster : 1];
   uint64_t full[S::kStages];
   uint64_t empty[S::kStages];
 };
@@ -80,21 +85,48 @@ struct DecodeArgs {
 };
 
 
-template <typename T, int D>
+// kCluster = false: stream-K pieces from the work tables, partials merged
+//   through global memory by the CTA that finishes a ring last.
+// kCluster = true: one ring per cluster of v.cluster_size CTAs, each taking an
+//   equal key range; partials go to the leader CTA's shared memory and one
+//   cluster barrier replaces the global publish/merge (small batches, where
+//   that hand-off dominates the step).
+template <typename T, int D, bool kCluster>
 __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     decode_split_kernel(const DecodeArgs a) {
   using S = DecodeShape<T, D>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  DecodeSmem<T, D> &sm = *reinterpret_cast<DecodeSmem<T, D> *>(smem_raw);
+  DecodeSmem<T, D, kCluster> &sm = *reinterpret_cast<DecodeSmem<T, D, kCluster> *>(smem_raw);
   const DeviceView &v = a.v;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int p_begin = v.cta_piece[blockIdx.x];
-  const int p_end = v.cta_piece[blockIdx.x + 1];
-  // the work plan is written once when the state is built, so this CTA's
-  // first piece can be fetched before the grid-dependency wait below
-  const DecodePiece first_piece = v.pieces[p_begin];
+  int p_begin = 0, p_end = 1, rank = 0;
+  // The work plan is written once when the state is built, so this CTA's
+  // first piece can be fetched before the grid-dependency wait below.
+  DecodePiece first_piece;
+  if constexpr (kCluster) {
+    const int C = v.cluster_size;
+    rank = (int)(blockIdx.x % (unsigned)C);
+    const int ring = (int)(blockIdx.x / (unsigned)C);
+    const int b = ring / v.H, h = ring % v.H;
+    const int P = v.plen[b];
+    const int len = P + v.W;
+    const int per = (len + C - 1) / C;
+    first_piece.row0 = (int64_t)v.H * v.slot_base[b] + (int64_t)h * len;
+    first_piece.b = b;
+    first_piece.h = h;
+    first_piece.key_begin = min(rank * per, len);
+    first_piece.key_end = min((rank + 1) * per, len);
+    first_piece.plen = P;
+    first_piece.first = 0;
+    first_piece.count = C;
+    first_piece.cta = (int)blockIdx.x;
+  } else {
+    p_begin = v.cta_piece[blockIdx.x];
+    p_end = v.cta_piece[blockIdx.x + 1];
+    first_piece = v.pieces[p_begin];
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
@@ -104,6 +136,11 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     fence_mbar_init();
   }
   __syncthreads();
+  // Cluster variant: every thread arrives once at the start; consumers wait
+  // on that phase before their first distributed-shared-memory store, so no
+  // CTA writes into a peer that has not started.  (The producer warp arrives
+  // and later exits; a cluster barrier waits only for non-exited threads.)
+  if constexpr (kCluster) cluster_arrive_relaxed();
 
   // Prompt rows (slots < P_b) are written only by the prefill's cache fill
   // or by the caller, never by a kernel that lets its dependents start early
@@ -312,20 +349,38 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     float M = -INFINITY;
 #pragma unroll
     for (int gg = 0; gg < S::kGroups; ++gg) M = fmaxf(M, sm.red_m[gg]);
-    for (int e = tid; e < D; e += 128) {
-      float acc = 0.f;
-      if (M != -INFINITY)
+    float acc_e = 0.f;  // this thread's output element (tid < D)
+    if (tid < D && M != -INFINITY)
 #pragma unroll
-        for (int gg = 0; gg < S::kGroups; ++gg)
-          acc = fmaf(sm.red_o[gg][e], exp2f(sm.red_m[gg] - M), acc);
-      v.part_o[(int64_t)p * D + e] = acc;
+      for (int gg = 0; gg < S::kGroups; ++gg)
+        acc_e = fmaf(sm.red_o[gg][tid], exp2f(sm.red_m[gg] - M), acc_e);
+    float L = 0.f;
+    if (tid == 0 && M != -INFINITY)
+      for (int gg = 0; gg < S::kGroups; ++gg) L = fmaf(sm.red_l[gg], exp2f(sm.red_m[gg] - M), L);
+    if constexpr (kCluster) {
+      // -------- hand the partial to the leader CTA's shared memory, then one
+      // cluster barrier (release/acquire) and the leader merges
+      cluster_wait_acquire();  // the start-of-kernel phase
+      if (tid < D) st_cluster_f32(map_to_rank(&sm.cl_o[rank][tid], 0), acc_e);
+      if (tid == 0) st_cluster_f32x2(map_to_rank(&sm.cl_ml[rank], 0), M, L);
+      cluster_arrive_release();
+      cluster_wait_acquire();
+      if (rank == 0 && tid < D) {
+        const int C = v.cluster_size;
+        float Mg = -INFINITY;
+        for (int r = 0; r < C; ++r) Mg = fmaxf(Mg, sm.cl_ml[r].x);
+        float Lg = 0.f, acc = 0.f;
+        for (int r = 0; r < C; ++r) {
+          const float wgt = exp2f(sm.cl_ml[r].x - Mg);  // 0 for an empty range
+          Lg = fmaf(wgt, sm.cl_ml[r].y, Lg);
+          acc = fmaf(wgt, sm.cl_o[r][tid], acc);
+        }
+        ((T *)a.out)[((int64_t)pc.b * v.H + pc.h) * D + tid] = from_float<T>(acc / Lg);
+      }
+      continue;  // a cluster CTA has exactly one piece
     }
-    if (tid == 0) {
-      float L = 0.f;
-      if (M != -INFINITY)
-        for (int gg = 0; gg < S::kGroups; ++gg) L = fmaf(sm.red_l[gg], exp2f(sm.red_m[gg] - M), L);
-      v.part_ml[p] = make_float2(M, L);
-    }
+    if (tid < D) v.part_o[(int64_t)p * D + tid] = acc_e;
+    if (tid == 0) v.part_ml[p] = make_float2(M, L);
     // -------- publish the partial; the last piece of this (b, h) merges.
     // The barrier orders every thread's partial stores before thread 0's
     // acq_rel atomic, whose release makes them visible device-wide and whose
@@ -389,45 +444,92 @@ __global__ void advance_kernel(int64_t *t, int B) {
   if (b < B) t[b] += 1;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kCluster>
+cudaError_t set_smem_attr() {
+  const int smem = (int)sizeof(DecodeSmem<T, D, kCluster>);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<T, D, kCluster>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && kCluster)
+    e = cudaFuncSetAttribute(decode_split_kernel<T, D, kCluster>,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <typename T, int D, bool kCluster>
 cudaError_t launch_decode_t(const DeviceView &v, const void *q, const void *k_new,
                             const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
                             bool pdl) {
   using S = DecodeShape<T, D>;
-  const int smem = (int)sizeof(DecodeSmem<T, D>);
-  static bool attr_set = false;  // per (T, D) instantiation
+  static bool attr_set = false;  // per instantiation; also set when the state is built
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<T, D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_attr<T, D, kCluster>();
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   DecodeArgs a{v, q, k_new, v_new, kc, vc, out};
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(v.decode_grid);
+  lc.gridDim = dim3(kCluster ? v.B * v.H * v.cluster_size : v.decode_grid);
   lc.blockDim = dim3(S::kThreads);
-  lc.dynamicSmemBytes = smem;
+  lc.dynamicSmemBytes = sizeof(DecodeSmem<T, D, kCluster>);
   lc.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  int na = 1;
+  if (kCluster) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)v.cluster_size;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    na = 2;
+  }
   lc.attrs = attr;
-  lc.numAttrs = 1;
-  return cudaLaunchKernelEx(&lc, decode_split_kernel<T, D>, a);
+  lc.numAttrs = na;
+  return cudaLaunchKernelEx(&lc, decode_split_kernel<T, D, kCluster>, a);
+}
+
+template <typename T, int D>
+cudaError_t launch_decode_d(const DeviceView &v, const void *q, const void *k_new,
+                            const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
+                            bool pdl) {
+  return v.cluster_size > 0
+             ? launch_decode_t<T, D, true>(v, q, k_new, v_new, kc, vc, out, s, pdl)
+             : launch_decode_t<T, D, false>(v, q, k_new, v_new, kc, vc, out, s, pdl);
 }
 
 template <typename T, int D>
 int ctas_per_sm_t() {
   using S = DecodeShape<T, D>;
-  const int smem = (int)sizeof(DecodeSmem<T, D>);
-  if (cudaFuncSetAttribute(decode_split_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return 1;
+  if (set_smem_attr<T, D, false>() != cudaSuccess) return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<T, D>, S::kThreads,
-                                                    smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_split_kernel<T, D, false>,
+                                                    S::kThreads,
+                                                    sizeof(DecodeSmem<T, D, false>)) !=
+          cudaSuccess ||
       n < 1)
     return 1;
+  return n;
+}
+
+// Clusters of `cluster` CTAs that can be resident at once (0 if unsupported).
+template <typename T, int D>
+int max_clusters_t(int cluster) {
+  using S = DecodeShape<T, D>;
+  if (set_smem_attr<T, D, true>() != cudaSuccess) return 0;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(cluster * 1024);
+  lc.blockDim = dim3(S::kThreads);
+  lc.dynamicSmemBytes = sizeof(DecodeSmem<T, D, true>);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_split_kernel<T, D, true>, &lc) != cudaSuccess)
+    return 0;
   return n;
 }
 
@@ -438,11 +540,11 @@ cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
                           bool pdl) {
   if (v.dtype == RSWA_BF16) {
     if (v.D == 128)
-      return launch_decode_t<__nv_bfloat16, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
-    return launch_decode_t<__nv_bfloat16, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+      return launch_decode_d<__nv_bfloat16, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+    return launch_decode_d<__nv_bfloat16, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
   }
-  if (v.D == 128) return launch_decode_t<float, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
-  return launch_decode_t<float, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+  if (v.D == 128) return launch_decode_d<float, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+  return launch_decode_d<float, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
 }
 
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s) {
@@ -456,6 +558,13 @@ cudaError_t launch_advance(const DeviceView &v, cudaStream_t s) {
   lc.attrs = attr;
   lc.numAttrs = 1;
   return cudaLaunchKernelEx(&lc, advance_kernel, v.t, v.B);
+}
+
+int decode_max_clusters(int dtype, int head_dim, int cluster) {
+  if (dtype == RSWA_BF16)
+    return head_dim == 128 ? max_clusters_t<__nv_bfloat16, 128>(cluster)
+                           : max_clusters_t<__nv_bfloat16, 64>(cluster);
+  return head_dim == 128 ? max_clusters_t<float, 128>(cluster) : max_clusters_t<float, 64>(cluster);
 }
 
 int decode_ctas_per_sm(int dtype, int head_dim) {

@@ -81,6 +81,7 @@ struct DeviceView {
   float *part_o;
   int decode_grid;
   int n_pieces;
+  int cluster_size;  // > 0: decode runs one ring per cluster of this many CTAs
   int64_t total_tokens;  // sum P_b
   int total_tiles;       // sum ceil(P_b / kPrefillTile)
   int total_tiles64;     // sum ceil(P_b / kSimtTile)
@@ -128,6 +129,8 @@ cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int6
 
 // Resident decode CTAs per SM for (dtype, head_dim); used by the planner.
 int decode_ctas_per_sm(int dtype, int head_dim);
+// Clusters of `cluster` decode CTAs that can be resident at once (0: none).
+int decode_max_clusters(int dtype, int head_dim, int cluster);
 
 // Host-side helpers of the planner (rswa_api.cu).
 bool config_ok(const rswa_config *c, const int64_t *plen);

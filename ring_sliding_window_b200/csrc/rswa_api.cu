@@ -2,6 +2,7 @@
 // layout, and the exported C entry points declared in include/rswa.h.
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -179,6 +180,29 @@ namespace {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Decode split for this batch: 0 = stream-K pieces merged through global
+// memory; C > 0 = one ring per cluster of C CTAs merged through distributed
+// shared memory.  The cluster form is used when every ring's cluster can be
+// resident at once (small batches, where the global hand-off dominates).
+// RSWA_DECODE_SPLIT=streamk|cluster overrides the choice (the cluster form
+// still needs the clusters to fit).
+int choose_cluster_size(const rswa_config *c, const int64_t *plen) {
+  const char *env = getenv("RSWA_DECODE_SPLIT");
+  const bool force_streamk = env && strcmp(env, "streamk") == 0;
+  const bool force_cluster = env && strcmp(env, "cluster") == 0;
+  if (force_streamk) return 0;
+  int64_t max_len = 0;
+  for (int b = 0; b < c->batch; ++b) max_len = std::max<int64_t>(max_len, plen[b] + c->window);
+  int C = (int)std::min<int64_t>(16, std::max<int64_t>(2, (max_len + 63) / 64));
+  const int64_t rings = (int64_t)c->batch * c->num_heads;
+  for (; C >= 2; C /= 2) {
+    const int fit = decode_max_clusters(c->dtype, c->head_dim, C);
+    if (fit >= rings) break;
+    if (!force_cluster) return 0;
+  }
+  return C >= 2 ? C : 0;
+}
+
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
 rswa_status from_cuda(cudaError_t e) {
@@ -306,6 +330,7 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   v.part_o = (float *)(w + s->ws.part_o);
   v.decode_grid = s->plan.grid;
   v.n_pieces = s->plan.n_pieces;
+  v.cluster_size = choose_cluster_size(cfg, prefill_len);
   v.total_tokens = tb[B];
   v.total_tiles = tl[B];
   v.total_tiles64 = tl64[B];
@@ -404,6 +429,14 @@ rswa_status rswa_get_ring(const rswa_state *s, int64_t *n_generated, int32_t *ri
     if (ring_pos) ring_pos[b] = (int32_t)(t[(size_t)b] < W ? 0 : t[(size_t)b] % W);
     if (cache_len) cache_len[b] = s->plen[(size_t)b] + std::min(t[(size_t)b], W);
   }
+  return RSWA_OK;
+}
+
+rswa_status rswa_decode_launch_shape(const rswa_state *s, int32_t *grid, int32_t *cluster_size) {
+  if (!s) return RSWA_EINVAL;
+  const int C = s->dv.cluster_size;
+  if (grid) *grid = C > 0 ? s->cfg.batch * s->cfg.num_heads * C : s->dv.decode_grid;
+  if (cluster_size) *cluster_size = C;
   return RSWA_OK;
 }
 

@@ -31,6 +31,7 @@ EXPORTED = (
     "rswa_cache_offset", "rswa_prefill", "rswa_decode_step", "rswa_advance", "rswa_reset_ring",
     "rswa_ngram_mask", "rswa_get_ring", "rswa_check_device_error", "rswa_status_string",
     "rswa_decode_step_noalloc", "rswa_last_cuda_error", "rswa_debug_inject_fault",
+    "rswa_decode_launch_shape",
 )
 RSWA_FAULT_DROP_DECODE_COPIES = 1
 RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -79,6 +80,7 @@ lib.rswa_ngram_mask.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, c
                                 ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp]
 lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
+lib.rswa_decode_launch_shape.argtypes = [_vp, _i32p, _i32p]
 lib.rswa_decode_step_noalloc.argtypes = [_cfgp, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.rswa_decode_step_noalloc.restype = ctypes.c_int
 lib.rswa_debug_inject_fault.argtypes = [_vp, ctypes.c_int32, _vp]
@@ -89,7 +91,7 @@ lib.rswa_status_string.argtypes = [ctypes.c_int]
 lib.rswa_status_string.restype = ctypes.c_char_p
 for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_decode_step",
            "rswa_advance", "rswa_reset_ring", "rswa_ngram_mask", "rswa_get_ring",
-           "rswa_check_device_error"):
+           "rswa_check_device_error", "rswa_decode_launch_shape"):
     getattr(lib, _n).restype = ctypes.c_int
 
 
@@ -196,6 +198,14 @@ def rswa_get_ring(state, batch: int, stream=None):
     return list(n), list(rp), list(cl)
 
 
+def rswa_decode_launch_shape(state):
+    """(grid, cluster_size) of this state's decode launches; cluster_size 0 = stream-K split."""
+    g, c = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib.rswa_decode_launch_shape(state, ctypes.byref(g), ctypes.byref(c)),
+           "rswa_decode_launch_shape")
+    return int(g.value), int(c.value)
+
+
 def rswa_check_device_error(state, stream=None) -> int:
     """Returns the status (does not raise): RSWA_OK, RSWA_ETIMEOUT or RSWA_EDEVICE."""
     return int(lib.rswa_check_device_error(state, _stream(stream)))
@@ -273,3 +283,6 @@ class State:
 
     def check(self, stream=None) -> int:
         return rswa_check_device_error(self.handle, stream)
+
+    def decode_launch_shape(self):
+        return rswa_decode_launch_shape(self.handle)

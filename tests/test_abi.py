@@ -84,6 +84,7 @@ def test_null_state_and_ngram_args_rejected(rswa):
     assert lib.rswa_advance(None, None) == rswa.RSWA_EINVAL
     assert lib.rswa_reset_ring(None, None) == rswa.RSWA_EINVAL
     assert lib.rswa_check_device_error(None, None) == rswa.RSWA_EINVAL
+    assert lib.rswa_decode_launch_shape(None, None, None) == rswa.RSWA_EINVAL
     assert lib.rswa_state_destroy(None) == rswa.RSWA_EINVAL
     assert lib.rswa_cache_offset(None, 0, 0, 0) == -1
     # rows < 0, vocab < 1, n < 1, ld < vocab, hist_ld < window, null logits

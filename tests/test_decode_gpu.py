@@ -48,11 +48,20 @@ FULL_RUN_CASES = [
 ]
 
 
+@pytest.mark.parametrize("split", ["streamk", "cluster"])
 @pytest.mark.parametrize("w", FULL_RUN_CASES, ids=lambda w: w.name)
-def test_decode_full_run_vs_oracle_ring(w):
+def test_decode_full_run_vs_oracle_ring(w, split, monkeypatch):
     """Every step of the run against the oracle's three-phase ring simulation;
-    ring counters and cache contents bit-exact after every step."""
+    ring counters and cache contents bit-exact after every step.  Both decode
+    splits run: stream-K ranges merged through the workspace, and one cluster
+    per ring merged through distributed shared memory."""
+    monkeypatch.setenv("RSWA_DECODE_SPLIT", split)
     st = _state(w)
+    grid, csize = st.decode_launch_shape()
+    if split == "streamk":
+        assert csize == 0
+    else:
+        assert csize >= 2 and grid == w.batch * w.heads * csize
     ins, _ = _prefill_all(st, w)
     sl = seq_slices(w.prefill_lens)
     model = oracle.RingModel(w.prefill_lens, w.window, w.layers, w.heads, w.head_dim)
