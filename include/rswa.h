@@ -123,6 +123,60 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
                               void *const *v_cache, void *workspace, size_t workspace_size,
                               void *stream, rswa_state **out);
 
+/* ------------------------------------------------------------------------
+ * Token pool and continuous batching [§三: serving with a page size of one
+ * token].  Each request owns P_b + W cache slots for its whole life, so a
+ * serving process keeps one K/V pool per layer and gives each joining request
+ * one contiguous slot range, freed when the request leaves.  Requests join
+ * and leave between decode steps: the caller builds a state over the requests
+ * running now (rswa_state_create_pooled, with each request's slot base and its
+ * current n_generated from rswa_get_ring of the previous state) and destroys
+ * the old one; a joining request's prompt is filled by rswa_prefill of a
+ * state over the joining requests alone, pointing at the same pool.
+ * ------------------------------------------------------------------------ */
+typedef struct rswa_pool rswa_pool;
+
+/* Host-side allocator of slot ranges in a pool of `capacity` slots
+ * (1 <= capacity < 2^40).  Allocation is first fit: the lowest base with
+ * enough free slots after it.  Freed ranges merge with free neighbours.
+ * Thread-safe.  No device memory is involved. */
+rswa_status rswa_pool_create(int64_t capacity, rswa_pool **out);
+rswa_status rswa_pool_destroy(rswa_pool *pool);
+/* `slots` >= 1 contiguous slots; *base receives the first.  RSWA_ENOMEM when
+ * no free range is long enough (the pool is unchanged). */
+rswa_status rswa_pool_alloc(rswa_pool *pool, int64_t slots, int64_t *base);
+/* Free the range that rswa_pool_alloc returned at `base`; RSWA_EINVAL if
+ * `base` is not the start of an allocated range. */
+rswa_status rswa_pool_free(rswa_pool *pool, int64_t base);
+/* Any pointer may be NULL: free slots, longest free range, number of free
+ * ranges, number of allocated ranges. */
+rswa_status rswa_pool_stats(const rswa_pool *pool, int64_t *free_slots, int64_t *largest_free,
+                            int32_t *n_free_ranges, int32_t *n_allocated);
+/* Capacity in slots, or -1 for NULL. */
+int64_t rswa_pool_capacity(const rswa_pool *pool);
+
+/* Bytes of ONE pool cache buffer (K or V) of ONE layer holding `pool_slots`
+ * slots: pool_slots * H * d * elem_size.  0 if invalid.  The batch field of
+ * cfg is ignored. */
+size_t rswa_pool_cache_bytes(const rswa_config *cfg, int64_t pool_slots);
+
+/* As rswa_state_create, for requests placed anywhere in a pool:
+ *  slot_base  : host [B] or NULL.  Request b's cache is slots
+ *               [slot_base[b], slot_base[b] + P_b + W) of the pool, laid out
+ *               head-major like the packed layout with S_b = slot_base[b]:
+ *                 element offset of (b, h, slot, e) =
+ *                     (H * slot_base[b] + h * (P_b + W) + slot) * d + e.
+ *               NULL: packed back to back (pool_slots is then ignored).
+ *  pool_slots : slots each cache buffer holds (rswa_pool_cache_bytes).
+ * Returns RSWA_EINVAL if a range leaves [0, pool_slots) or two requests'
+ * ranges overlap.  The workspace size is rswa_workspace_bytes(cfg,
+ * prefill_len), as for a packed batch. */
+rswa_status rswa_state_create_pooled(const rswa_config *cfg, const int64_t *prefill_len,
+                                     const int64_t *n_generated, const int64_t *slot_base,
+                                     int64_t pool_slots, void *const *k_cache,
+                                     void *const *v_cache, void *workspace, size_t workspace_size,
+                                     void *stream, rswa_state **out);
+
 /* Free the host-side state.  Device memory stays the caller's. */
 rswa_status rswa_state_destroy(rswa_state *state);
 

@@ -74,7 +74,7 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
   if (dev < 0) return RSWA_ECUDA;
 
   const DecodePlan plan =
-      plan_decode(cfg, prefill_len, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+      plan_decode(cfg, prefill_len, nullptr, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
   const WsLayout ws = layout_ws(cfg, prefill_len, plan);
   if (ws.total > kNoAllocScratchBytes) return RSWA_ENOMEM;  // batch too large for the array
 

@@ -93,6 +93,8 @@ struct DeviceView {
 struct rswa_state {
   rswa_config cfg;
   std::vector<int64_t> plen;
+  std::vector<int64_t> slot_base;  // first cache slot of each request
+  int64_t pool_slots;              // slots the caches hold (per layer, K or V)
   std::vector<void *> k_cache, v_cache;
   std::vector<uint8_t> layer_ready;  // prefilled or resumed
   void *workspace;
@@ -136,7 +138,10 @@ int decode_max_clusters(int dtype, int head_dim, int cluster);
 bool config_ok(const rswa_config *c, const int64_t *plen);
 int current_device();
 int sm_count(int dev);
-DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, int ctas_per_sm);
+// slot_base: host [B] first cache slot of each request, or NULL for requests
+// packed back to back in batch order.
+DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, const int64_t *slot_base,
+                       int num_sms, int ctas_per_sm);
 WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &p);
 
 }  // namespace rswa

@@ -60,8 +60,12 @@ int sm_count(int dev) {
 }
 
 // Equal contiguous ranges of the flattened (b, h, key) rows, one per CTA.
-DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, int ctas_per_sm) {
+DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, const int64_t *slot_base,
+                       int num_sms, int ctas_per_sm) {
   const int B = c->batch, H = c->num_heads, W = c->window;
+  std::vector<int64_t> base((size_t)B, 0);
+  for (int b = 0; b < B; ++b)
+    base[(size_t)b] = slot_base ? slot_base[b] : (b ? base[(size_t)b - 1] + plen[b - 1] + W : 0);
   std::vector<int64_t> seg_start((size_t)B * H + 1, 0);
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < H; ++h)
@@ -87,7 +91,7 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, int num_sms, i
       DecodePiece pc;
       pc.b = (int32_t)(seg / (size_t)H);
       pc.h = (int32_t)(seg % (size_t)H);
-      pc.row0 = seg_start[seg];  // rings are laid out back to back in (b, h) order
+      pc.row0 = (int64_t)H * base[(size_t)pc.b] + (int64_t)pc.h * (plen[pc.b] + W);
       pc.key_begin = (int32_t)(r0 - seg_start[seg]);
       pc.key_end = (int32_t)(e - seg_start[seg]);
       pc.plen = (int32_t)plen[pc.b];
@@ -227,18 +231,51 @@ size_t rswa_workspace_bytes(const rswa_config *cfg, const int64_t *prefill_len) 
   if (!config_ok(cfg, prefill_len)) return 0;
   const int dev = current_device();
   if (dev < 0) return 0;
-  const DecodePlan p =
-      plan_decode(cfg, prefill_len, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+  const DecodePlan p = plan_decode(cfg, prefill_len, nullptr, sm_count(dev),
+                                   decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
   return layout_ws(cfg, prefill_len, p).total;
+}
+
+size_t rswa_pool_cache_bytes(const rswa_config *cfg, int64_t pool_slots) {
+  if (!cfg || pool_slots < 1) return 0;
+  std::vector<int64_t> one(1, 0);
+  rswa_config c1 = *cfg;
+  c1.batch = 1;
+  if (!config_ok(&c1, one.data())) return 0;
+  if ((int64_t)cfg->num_heads * pool_slots >= (int64_t(1) << 40)) return 0;
+  return (size_t)pool_slots * (size_t)cfg->num_heads * (size_t)cfg->head_dim * elem_size(cfg);
 }
 
 rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len,
                               const int64_t *n_generated, void *const *k_cache,
                               void *const *v_cache, void *workspace, size_t workspace_size,
                               void *stream, rswa_state **out) {
+  return rswa_state_create_pooled(cfg, prefill_len, n_generated, nullptr, 0, k_cache, v_cache,
+                                  workspace, workspace_size, stream, out);
+}
+
+rswa_status rswa_state_create_pooled(const rswa_config *cfg, const int64_t *prefill_len,
+                                     const int64_t *n_generated, const int64_t *slot_base,
+                                     int64_t pool_slots, void *const *k_cache,
+                                     void *const *v_cache, void *workspace, size_t workspace_size,
+                                     void *stream, rswa_state **out) {
   if (!out) return RSWA_EINVAL;
   *out = nullptr;
   if (!config_ok(cfg, prefill_len) || !k_cache || !v_cache || !workspace) return RSWA_EINVAL;
+  if (slot_base) {
+    // every request's range inside the pool, no two ranges overlapping
+    if (pool_slots < 1 || (int64_t)cfg->num_heads * pool_slots >= (int64_t(1) << 40))
+      return RSWA_EINVAL;
+    std::vector<std::pair<int64_t, int64_t>> r((size_t)cfg->batch);
+    for (int b = 0; b < cfg->batch; ++b) {
+      const int64_t e = slot_base[b] + prefill_len[b] + cfg->window;
+      if (slot_base[b] < 0 || e > pool_slots) return RSWA_EINVAL;
+      r[(size_t)b] = {slot_base[b], e};
+    }
+    std::sort(r.begin(), r.end());
+    for (size_t i = 1; i < r.size(); ++i)
+      if (r[i].first < r[i - 1].second) return RSWA_EINVAL;
+  }
   if (((uintptr_t)workspace & 255u) != 0) return RSWA_EINVAL;
   for (int l = 0; l < cfg->num_layers; ++l)
     if (!k_cache[l] || !v_cache[l] || !aligned16(k_cache[l]) || !aligned16(v_cache[l]))
@@ -254,6 +291,13 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   s->cfg = *cfg;
   if (s->cfg.scale == 0.f) s->cfg.scale = 1.0f / sqrtf((float)cfg->head_dim);
   s->plen.assign(prefill_len, prefill_len + cfg->batch);
+  s->slot_base.assign((size_t)cfg->batch, 0);
+  s->pool_slots = 0;
+  for (int b = 0; b < cfg->batch; ++b) {
+    s->slot_base[(size_t)b] = slot_base ? slot_base[b] : s->pool_slots;
+    if (!slot_base) s->pool_slots += prefill_len[b] + cfg->window;
+  }
+  if (slot_base) s->pool_slots = pool_slots;
   s->k_cache.assign(k_cache, k_cache + cfg->num_layers);
   s->v_cache.assign(v_cache, v_cache + cfg->num_layers);
   s->layer_ready.assign((size_t)cfg->num_layers, n_generated ? 1 : 0);
@@ -261,7 +305,8 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
   s->workspace_size = workspace_size;
   s->device = dev;
   s->num_sms = sm_count(dev);
-  s->plan = plan_decode(cfg, prefill_len, s->num_sms, decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+  s->plan = plan_decode(cfg, prefill_len, s->slot_base.data(), s->num_sms,
+                        decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
   s->ws = layout_ws(cfg, prefill_len, s->plan);
   if (workspace_size < s->ws.total) {
     delete s;
@@ -283,7 +328,7 @@ rswa_status rswa_state_create(const rswa_config *cfg, const int64_t *prefill_len
     t[b] = n_generated ? n_generated[b] : 0;
     t[B + b] = t[b];  // reset copy
     pl[b] = (int32_t)prefill_len[b];
-    sb[b + 1] = sb[b] + prefill_len[b] + cfg->window;
+    sb[b] = s->slot_base[(size_t)b];
     tb[b + 1] = tb[b] + prefill_len[b];
     tl[b + 1] = tl[b] + (int32_t)((prefill_len[b] + kPrefillTile - 1) / kPrefillTile);
     tl64[b + 1] = tl64[b] + (int32_t)((prefill_len[b] + kSimtTile - 1) / kSimtTile);
@@ -349,8 +394,7 @@ int64_t rswa_cache_offset(const rswa_state *s, int32_t b, int32_t h, int64_t slo
   if (!s || b < 0 || b >= s->cfg.batch || h < 0 || h >= s->cfg.num_heads) return -1;
   const int64_t P = s->plen[(size_t)b];
   if (slot < 0 || slot >= P + s->cfg.window) return -1;
-  int64_t base = 0;
-  for (int i = 0; i < b; ++i) base += s->plen[(size_t)i] + s->cfg.window;
+  const int64_t base = s->slot_base[(size_t)b];
   return ((int64_t)s->cfg.num_heads * base + (int64_t)h * (P + s->cfg.window) + slot) *
          s->cfg.head_dim;
 }

@@ -31,7 +31,9 @@ EXPORTED = (
     "rswa_cache_offset", "rswa_prefill", "rswa_decode_step", "rswa_advance", "rswa_reset_ring",
     "rswa_ngram_mask", "rswa_get_ring", "rswa_check_device_error", "rswa_status_string",
     "rswa_decode_step_noalloc", "rswa_last_cuda_error", "rswa_debug_inject_fault",
-    "rswa_decode_launch_shape",
+    "rswa_decode_launch_shape", "rswa_pool_create", "rswa_pool_destroy", "rswa_pool_alloc",
+    "rswa_pool_free", "rswa_pool_stats", "rswa_pool_capacity", "rswa_pool_cache_bytes",
+    "rswa_state_create_pooled",
 )
 RSWA_FAULT_DROP_DECODE_COPIES = 1
 RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -81,6 +83,18 @@ lib.rswa_ngram_mask.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, c
 lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
 lib.rswa_decode_launch_shape.argtypes = [_vp, _i32p, _i32p]
+lib.rswa_pool_create.argtypes = [ctypes.c_int64, ctypes.POINTER(_vp)]
+lib.rswa_pool_destroy.argtypes = [_vp]
+lib.rswa_pool_alloc.argtypes = [_vp, ctypes.c_int64, _i64p]
+lib.rswa_pool_free.argtypes = [_vp, ctypes.c_int64]
+lib.rswa_pool_stats.argtypes = [_vp, _i64p, _i64p, _i32p, _i32p]
+lib.rswa_pool_capacity.argtypes = [_vp]
+lib.rswa_pool_capacity.restype = ctypes.c_int64
+lib.rswa_pool_cache_bytes.argtypes = [_cfgp, ctypes.c_int64]
+lib.rswa_pool_cache_bytes.restype = ctypes.c_size_t
+lib.rswa_state_create_pooled.argtypes = [_cfgp, _i64p, _i64p, _i64p, ctypes.c_int64,
+                                         ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp,
+                                         ctypes.c_size_t, _vp, ctypes.POINTER(_vp)]
 lib.rswa_decode_step_noalloc.argtypes = [_cfgp, _i64p, _i64p, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.rswa_decode_step_noalloc.restype = ctypes.c_int
 lib.rswa_debug_inject_fault.argtypes = [_vp, ctypes.c_int32, _vp]
@@ -91,7 +105,9 @@ lib.rswa_status_string.argtypes = [ctypes.c_int]
 lib.rswa_status_string.restype = ctypes.c_char_p
 for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_decode_step",
            "rswa_advance", "rswa_reset_ring", "rswa_ngram_mask", "rswa_get_ring",
-           "rswa_check_device_error", "rswa_decode_launch_shape"):
+           "rswa_check_device_error", "rswa_decode_launch_shape", "rswa_pool_create",
+           "rswa_pool_destroy", "rswa_pool_alloc", "rswa_pool_free", "rswa_pool_stats",
+           "rswa_state_create_pooled"):
     getattr(lib, _n).restype = ctypes.c_int
 
 
@@ -149,6 +165,57 @@ def rswa_state_create(cfg, prefill_len, n_generated, k_cache, v_cache, workspace
                                ctypes.byref(out))
     _check(st, "rswa_state_create")
     return out
+
+
+def rswa_state_create_pooled(cfg, prefill_len, n_generated, slot_base, pool_slots, k_cache,
+                             v_cache, workspace, workspace_size, stream=None) -> ctypes.c_void_p:
+    kp = (ctypes.c_void_p * len(k_cache))(*[_ptr(t).value for t in k_cache])
+    vp = (ctypes.c_void_p * len(v_cache))(*[_ptr(t).value for t in v_cache])
+    out = ctypes.c_void_p()
+    st = lib.rswa_state_create_pooled(ctypes.byref(cfg), _i64(prefill_len),
+                                      None if n_generated is None else _i64(n_generated),
+                                      None if slot_base is None else _i64(slot_base),
+                                      int(pool_slots), kp, vp, _ptr(workspace),
+                                      int(workspace_size), _stream(stream), ctypes.byref(out))
+    _check(st, "rswa_state_create_pooled")
+    return out
+
+
+def rswa_pool_cache_bytes(cfg: rswa_config, pool_slots: int) -> int:
+    return int(lib.rswa_pool_cache_bytes(ctypes.byref(cfg), int(pool_slots)))
+
+
+def rswa_pool_create(capacity: int) -> ctypes.c_void_p:
+    out = ctypes.c_void_p()
+    _check(lib.rswa_pool_create(int(capacity), ctypes.byref(out)), "rswa_pool_create")
+    return out
+
+
+def rswa_pool_destroy(pool) -> None:
+    _check(lib.rswa_pool_destroy(pool), "rswa_pool_destroy")
+
+
+def rswa_pool_alloc(pool, slots: int) -> int:
+    base = ctypes.c_int64(0)
+    _check(lib.rswa_pool_alloc(pool, int(slots), ctypes.byref(base)), "rswa_pool_alloc")
+    return int(base.value)
+
+
+def rswa_pool_free(pool, base: int) -> None:
+    _check(lib.rswa_pool_free(pool, int(base)), "rswa_pool_free")
+
+
+def rswa_pool_stats(pool):
+    """(free_slots, largest_free_range, n_free_ranges, n_allocated)."""
+    f, lg = ctypes.c_int64(0), ctypes.c_int64(0)
+    nf, na = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib.rswa_pool_stats(pool, ctypes.byref(f), ctypes.byref(lg), ctypes.byref(nf),
+                               ctypes.byref(na)), "rswa_pool_stats")
+    return int(f.value), int(lg.value), int(nf.value), int(na.value)
+
+
+def rswa_pool_capacity(pool) -> int:
+    return int(lib.rswa_pool_capacity(pool))
 
 
 def rswa_state_destroy(state) -> None:
@@ -232,19 +299,30 @@ class State:
     """A batch's caches + workspace (torch-allocated) and its rswa_state."""
 
     def __init__(self, batch, num_layers, num_heads, head_dim, window, prefill_lens,
-                 dtype=torch.bfloat16, n_generated=None, scale=0.0, device="cuda", stream=None):
+                 dtype=torch.bfloat16, n_generated=None, scale=0.0, device="cuda", stream=None,
+                 pool=None, slot_base=None):
         self.cfg = make_config(batch, num_layers, num_heads, head_dim, window, dtype, scale)
         self.dtype = torch.bfloat16 if self.cfg.dtype == RSWA_BF16 else torch.float32
         self.prefill_lens = [int(p) for p in prefill_lens]
         self.B, self.L, self.H, self.d, self.W = batch, num_layers, num_heads, head_dim, window
-        cb = rswa_cache_bytes(self.cfg, self.prefill_lens)
         wb = rswa_workspace_bytes(self.cfg, self.prefill_lens)
-        if cb == 0 or wb == 0:
-            raise RswaError(RSWA_EINVAL, "rswa_cache_bytes/rswa_workspace_bytes")
+        if wb == 0:
+            raise RswaError(RSWA_EINVAL, "rswa_workspace_bytes")
+        self.workspace = torch.empty(wb, dtype=torch.uint8, device=device)
+        if pool is not None:
+            # requests placed in a TokenPool's caches at the given slot bases
+            self.k_cache, self.v_cache = pool.k_cache, pool.v_cache
+            self.slot_base = [int(x) for x in slot_base]
+            self.handle = rswa_state_create_pooled(self.cfg, self.prefill_lens, n_generated,
+                                                   self.slot_base, pool.capacity, self.k_cache,
+                                                   self.v_cache, self.workspace, wb, stream)
+            return
+        cb = rswa_cache_bytes(self.cfg, self.prefill_lens)
+        if cb == 0:
+            raise RswaError(RSWA_EINVAL, "rswa_cache_bytes")
         elems = cb // (2 if self.dtype == torch.bfloat16 else 4)
         self.k_cache = [torch.empty(elems, dtype=self.dtype, device=device) for _ in range(num_layers)]
         self.v_cache = [torch.empty(elems, dtype=self.dtype, device=device) for _ in range(num_layers)]
-        self.workspace = torch.empty(wb, dtype=torch.uint8, device=device)
         self.handle = rswa_state_create(self.cfg, self.prefill_lens, n_generated, self.k_cache,
                                         self.v_cache, self.workspace, wb, stream)
 
@@ -286,3 +364,48 @@ class State:
 
     def decode_launch_shape(self):
         return rswa_decode_launch_shape(self.handle)
+
+
+class TokenPool:
+    """One K/V pool per layer (torch-allocated) and the slot-range allocator:
+    requests join with `alloc(prefill_len)` and leave with `free(base)`; a
+    `State` over any set of live requests is built with `state(...)`."""
+
+    def __init__(self, capacity, num_layers, num_heads, head_dim, window, dtype=torch.bfloat16,
+                 device="cuda"):
+        self.capacity = int(capacity)
+        self.L, self.H, self.d, self.W = num_layers, num_heads, head_dim, window
+        self.dtype = dtype
+        cfg = make_config(1, num_layers, num_heads, head_dim, window, dtype)
+        cb = rswa_pool_cache_bytes(cfg, self.capacity)
+        if cb == 0:
+            raise RswaError(RSWA_EINVAL, "rswa_pool_cache_bytes")
+        elems = cb // (2 if dtype == torch.bfloat16 else 4)
+        self.k_cache = [torch.empty(elems, dtype=dtype, device=device) for _ in range(num_layers)]
+        self.v_cache = [torch.empty(elems, dtype=dtype, device=device) for _ in range(num_layers)]
+        self.handle = rswa_pool_create(self.capacity)
+
+    def alloc(self, prefill_len: int) -> int:
+        return rswa_pool_alloc(self.handle, int(prefill_len) + self.W)
+
+    def free(self, base: int) -> None:
+        rswa_pool_free(self.handle, base)
+
+    def stats(self):
+        return rswa_pool_stats(self.handle)
+
+    def state(self, prefill_lens, slot_bases, n_generated=None, stream=None, scale=0.0) -> State:
+        return State(len(prefill_lens), self.L, self.H, self.d, self.W, prefill_lens,
+                     dtype=self.dtype, n_generated=n_generated, scale=scale, stream=stream,
+                     pool=self, slot_base=slot_bases)
+
+    def close(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h:
+            rswa_pool_destroy(h)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
