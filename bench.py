@@ -474,7 +474,12 @@ def run_ours(args, rank, world, local_rank):
     also = []
     if world == 1 and args.also != "none":
         for name in args.also.split(","):
-            also.append(run_also(synth.workload(name), args, flush, s, hbm_peak, tc_peak))
+            if name == "continuous_batching":
+                also.append(run_continuous_batching(args, s, hbm_peak))
+            elif name == "ngram_topk":
+                also.append(run_ngram_topk(args, flush, s, hbm_peak))
+            else:
+                also.append(run_also(synth.workload(name), args, flush, s, hbm_peak, tc_peak))
             torch.cuda.empty_cache()
         line["also"] = also
 
@@ -485,6 +490,177 @@ def run_ours(args, rank, world, local_rank):
                                 "sample": f"{n} decode steps x {lps} layers of {w.name} from t=0 "
                                           f"(plus the n-gram ban) in {el:.1f} s"}
     return line
+
+
+def run_continuous_batching(args, s, hbm_peak, steps=64, churn_every=8, churn=4):
+    """Continuous batching on one token pool: the ragged-serving batch (64
+    requests, prefill_len U{1024..16384}, ring fill U{0..128}) placed in a
+    pool with 25 % headroom; every `churn_every` steps `churn` random requests
+    leave and as many new ones (same distributions) join, and the decode state
+    is rebuilt over the live requests.  Joining requests' caches hold random
+    values (their prefill is not timed: the prefill figures are measured
+    elsewhere).  Timed with CUDA events around the whole run, rebuilds
+    included; every input is larger than L2."""
+    import random
+    from ring_sliding_window_b200 import rswa
+    w = synth.workload("ragged_serving")
+    L, H, d, W = w.layers, w.heads, w.head_dim, w.window
+    rng = random.Random(synth.seed(w.cfg_id, 0, 950_000))
+    capacity = int(sum(P + W for P in w.prefill_lens) * 1.25)
+    pool = rswa.TokenPool(capacity, L, H, d, W, dtype=w.dtype)
+    for l in range(L):
+        g = torch.Generator(device="cuda").manual_seed(synth.seed(w.cfg_id, l, 950_001))
+        pool.k_cache[l].normal_(generator=g)
+        pool.v_cache[l].normal_(generator=g)
+    live = []  # [prefill_len, base, t]
+    order = list(range(w.batch))
+    rng.shuffle(order)
+    for b in order:
+        live.append([w.prefill_lens[b], pool.alloc(w.prefill_lens[b]), w.n_generated[b]])
+    bmax = w.batch
+    q = torch.randn(L, bmax, H, d, device="cuda").to(w.dtype)
+    kn, vn, out = torch.randn_like(q), torch.randn_like(q), torch.empty_like(q)
+
+    def build():
+        return pool.state([r[0] for r in live], [r[1] for r in live], n_generated=[r[2] for r in live],
+                          stream=s)
+
+    def step_bytes():
+        row = H * d * w.elem_bytes
+        return L * sum(2 * (P + min(t + 1, W)) * row + 6 * row for P, _, t in live)
+
+    def run(n_steps, st, record):
+        nbytes, rebuild_ms, skipped = 0, [], 0
+        for i in range(n_steps):
+            if i and i % churn_every == 0:
+                n, _, _ = st.ring(stream=s)  # waits for the queued steps
+                t0 = time.perf_counter()
+                for r, t in zip(live, n):
+                    r[2] = t
+                st.close()
+                for _ in range(churn):
+                    r = live.pop(rng.randrange(len(live)))
+                    pool.free(r[1])
+                for _ in range(churn):
+                    P = rng.randint(1024, 16384)
+                    try:
+                        live.append([P, pool.alloc(P), rng.randint(0, 128)])
+                    except rswa.RswaError:
+                        skipped += 1
+                st = build()
+                rebuild_ms.append((time.perf_counter() - t0) * 1e3)
+            B = len(live)
+            if record:
+                nbytes += step_bytes()
+            with torch.cuda.stream(s):
+                for l in range(L):
+                    st.decode_step(l, q[l, :B], kn[l, :B], vn[l, :B], out[l, :B], stream=s)
+                st.advance(stream=s)
+            for r in live:
+                r[2] += 1
+        return st, nbytes, rebuild_ms, skipped
+
+    st = build()
+    st, _, _, _ = run(max(args.warmup, churn_every + 1), st, False)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    st, nbytes, rebuild_ms, skipped = run(steps, st, True)
+    e1.record(s)
+    s.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert st.check() == 0
+    free, largest, n_free, n_alloc = pool.stats()
+    st.close()
+    pool.close()
+    return {"workload": "continuous_batching (ragged_serving requests in one token pool)",
+            "decode_steps_per_s": steps / (ms / 1e3), "ms_per_step": ms / steps,
+            "kv_read_gbs": nbytes / (ms / 1e3) / 1e9,
+            "frac_of_measured_hbm": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
+            "steps_timed": steps, "churn": f"{churn} leave + {churn} join every {churn_every} steps",
+            "rebuilds": len(rebuild_ms),
+            "rebuild_host_ms_mean": statistics.mean(rebuild_ms),
+            "rebuild_host_ms_max": max(rebuild_ms),
+            "rebuild": "frees, allocations, rswa_state_create_pooled (plan + table upload, "
+                       "synchronous), after the ring counters are read back",
+            "joins_refused_for_space": skipped,
+            "pool": {"capacity_slots": capacity, "free_slots": free, "largest_free": largest,
+                     "free_ranges": n_free, "requests": n_alloc}}
+
+
+def run_ngram_topk(args, flush, s, hbm_peak, reps=5, calls=16, nbuf=4):
+    """rswa_ngram_topk on the pages' sampling shape: 64 rows over the
+    129,280-token vocabulary, n = 35, window = 128 (the n-gram inputs of the
+    decode step), k = 1 (greedy) and k = 64 (with sampling).  Timed as a CUDA
+    graph of `calls` launches rotating over `nbuf` logits buffers (4 x 33 MB,
+    more than L2), events on the stream, median of `reps` replays: per-call
+    time.  Algorithmic bytes per call: the logits read once (rows x vocab x 4),
+    the histories and the outputs.  For context, one eager launch after an L2
+    flush, and the unfused pair rswa_ngram_mask + torch.topk timed the same
+    way, are reported too."""
+    from ring_sliding_window_b200 import rswa
+    rows, V, n, win = 64, synth.VOCAB, synth.NGRAM_SIZE, synth.NGRAM_WINDOW
+    logits, hist, _ = synth.ngram_inputs(rows, V, n, win, synth.seed(5, 0, 820_000))
+    bufs = [logits.cuda() for _ in range(nbuf)]
+    hist = hist.cuda()
+    u = torch.rand(rows, device="cuda")
+    out = {}
+
+    def graph_us(fn):
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for j in range(calls):
+                fn(bufs[j % nbuf])
+        torch.cuda.synchronize()
+        ms = []
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                g.replay()
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                g.replay()
+                e1.record(s)
+                ms.append((e0, e1))
+        s.synchronize()
+        del g
+        return statistics.median(a.elapsed_time(b) for a, b in ms) * 1e3 / calls
+
+    def eager_us(fn):
+        ms = []
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                fn(bufs[0])
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                fn(bufs[0])
+                e1.record(s)
+                ms.append((e0, e1))
+        s.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ms) * 1e3
+
+    for k in (1, 64):
+        idx = torch.empty(rows, k, dtype=torch.int32, device="cuda")
+        val = torch.empty(rows, k, device="cuda")
+        tok = torch.empty(rows, dtype=torch.int32, device="cuda")
+        samp = u if k > 1 else None
+        fused = lambda lg: rswa.rswa_ngram_topk(lg, hist, None, n, win, k, uniform=samp,
+                                                top_idx=idx, top_val=val, token=tok, stream=s)
+        unfused = lambda lg: (rswa.rswa_ngram_mask(lg, hist, None, n, win, stream=s),
+                              torch.topk(lg, k, dim=1))
+        us = graph_us(fused)
+        nbytes = rows * V * 4 + hist.numel() * 4 + rows * k * 8 + rows * 4
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[f"k{k}"] = {"us_per_call": us, "algorithmic_bytes": nbytes, "gbs": gbs,
+                        "frac_of_measured_hbm": gbs / hbm_peak,
+                        "eager_after_l2_flush_us": eager_us(fused),
+                        "sampling": "inverse CDF at a uniform per row" if samp is not None else "greedy",
+                        "unfused_mask_plus_torch_topk_us": graph_us(unfused)}
+    return {"workload": "ngram_topk (64 rows x 129,280 vocab, n=35, window=128)",
+            "timing": f"CUDA graph of {calls} calls over {nbuf} logits buffers (> L2)", **out}
 
 
 def run_also(w, args, flush, s, hbm_peak, tc_peak):
@@ -554,7 +730,8 @@ def main():
     ap.add_argument("--workload", default="single_page_decode")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
-    ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving")
+    ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving,"
+                                      "continuous_batching,ngram_topk")
     ap.add_argument("--also-steps", type=int, default=40)
     ap.add_argument("--skip-prefill-also", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

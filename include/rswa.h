@@ -242,6 +242,38 @@ rswa_status rswa_ngram_mask(float *logits, int64_t ld, const int32_t *history, i
                             const int32_t *hist_len, int32_t rows, int32_t vocab, int32_t n,
                             int32_t window, int32_t *device_error, void *stream);
 
+/* Fused n-gram ban + top-k selection, the step after the ban [§2.3: the
+ * banned tokens score -inf and the next token is chosen from the masked
+ * scores; greedy decoding at k = 1].
+ * For each row r < rows, with the banned set of rswa_ngram_mask (same
+ * history, hist_len, n, window and error rules), the masked row is
+ * x_j = -inf for banned j, logits[r, j] otherwise (NaN ranks as -inf).
+ * Columns are ordered by x_j descending, the lower column first among equal
+ * values; the first k of that order are written:
+ *  top_idx : device int32 [rows][k] (required);
+ *  top_val : device float [rows][k] or NULL -- x of those columns.
+ *  token   : device int32 [rows] or NULL -- the chosen token: with uniform
+ *            NULL, top_idx[r][0] (greedy); otherwise the inverse CDF at
+ *            uniform[r] of p_i proportional to exp((x_i - x_0) / temperature)
+ *            over the k columns: the first i whose running sum of p exceeds
+ *            uniform[r] * sum(p) (columns with x = -inf have p = 0).
+ *  uniform : device float [rows] in [0, 1), or NULL; temperature > 0 when set.
+ *  mask_in_place : nonzero also stores -inf into logits at the banned
+ *            columns, as rswa_ngram_mask does; zero leaves logits untouched.
+ * Limits: 1 <= k <= RSWA_TOPK_MAX and k <= vocab; vocab <= RSWA_TOPK_MAX_VOCAB;
+ * window <= 8192 (the history is staged in shared memory);
+ * ld >= vocab and ld a multiple of 4; logits 16-byte aligned (logits is
+ * read as float4 up to column ceil(vocab / 4) * 4 - 1 of each row).  A row
+ * whose history is invalid gets top_idx -1, top_val NaN and token -1, and the
+ * error bit in device_error.  Each row is read from HBM once. */
+#define RSWA_TOPK_MAX 64
+#define RSWA_TOPK_MAX_VOCAB 262144
+rswa_status rswa_ngram_topk(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                            const int32_t *hist_len, int32_t rows, int32_t vocab, int32_t n,
+                            int32_t window, int32_t k, int32_t mask_in_place,
+                            const float *uniform, float temperature, int32_t *top_idx,
+                            float *top_val, int32_t *token, int32_t *device_error, void *stream);
+
 /* Synchronises `stream`, then copies the ring counters to the host:
  *  n_generated : host [B] or NULL -- t_b;
  *  ring_pos    : host [B] or NULL -- the pages' ring_pos: 0 during warm-up,

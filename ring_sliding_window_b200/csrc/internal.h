@@ -55,6 +55,9 @@ struct DecodePlan {
   std::vector<int32_t> bh_piece;   // [B*H + 1]
 };
 
+constexpr int kTopkMax = 64;                 // largest k of rswa_ngram_topk
+constexpr int kTopkMaxVocab = 16 * 16384;    // 16 CTAs of 16,384 columns per row
+constexpr int kTopkMaxWindow = 8192;         // history staged in shared memory
 constexpr int kPrefillTile = 128;  // query rows per prefill tile (tensor-core kernel)
 constexpr int kSimtTile = 64;      // query rows per prefill tile (FP32 SIMT kernel)
 
@@ -115,6 +118,11 @@ cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
                           const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
                           bool pdl);
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s);
+cudaError_t launch_ngram_topk(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                              const int32_t *hist_len, int rows, int vocab, int n, int window,
+                              int k, int mask_in_place, const float *uniform, float temperature,
+                              int32_t *top_idx, float *top_val, int32_t *token, int *err,
+                              cudaStream_t s);
 cudaError_t launch_cache_fill(const DeviceView &v, const void *k, const void *vv, void *kc,
                               void *vc, cudaStream_t s);
 cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,

@@ -88,6 +88,16 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// 4-byte asynchronous global -> shared copy (no register staging); complete
+// with cp_async_wait_all() and a barrier before the data is read.
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -118,6 +128,25 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float x) {
 }
 __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float x, float y) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long x) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(x) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t x;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(x) : "r"(addr) : "memory");
+  return x;
+}
+__device__ __forceinline__ unsigned long long ld_cluster_u64(uint32_t addr) {
+  unsigned long long x;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(x) : "r"(addr) : "memory");
+  return x;
+}
+__device__ __forceinline__ uint32_t atom_add_cluster_u32(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v)
+               : "memory");
+  return old;
 }
 // Cluster-wide barrier over all non-exited threads (warp-uniform).
 __device__ __forceinline__ void cluster_arrive_release() {

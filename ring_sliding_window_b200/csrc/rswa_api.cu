@@ -457,6 +457,26 @@ rswa_status rswa_ngram_mask(float *logits, int64_t ld, const int32_t *history, i
                                 device_error, (cudaStream_t)stream));
 }
 
+rswa_status rswa_ngram_topk(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                            const int32_t *hist_len, int32_t rows, int32_t vocab, int32_t n,
+                            int32_t window, int32_t k, int32_t mask_in_place,
+                            const float *uniform, float temperature, int32_t *top_idx,
+                            float *top_val, int32_t *token, int32_t *device_error, void *stream) {
+  static_assert(RSWA_TOPK_MAX == kTopkMax && RSWA_TOPK_MAX_VOCAB == kTopkMaxVocab,
+                "header limits match the kernel");
+  if (rows < 0 || vocab < 1 || vocab > kTopkMaxVocab || n < 1 || window < 0) return RSWA_EINVAL;
+  if (k < 1 || k > kTopkMax || k > vocab) return RSWA_EINVAL;
+  if (ld < vocab || (ld & 3) != 0 || hist_ld < window || window > kTopkMaxWindow)
+    return RSWA_EINVAL;
+  if (uniform && !(temperature > 0.f && isfinite(temperature))) return RSWA_EINVAL;
+  if (rows == 0) return RSWA_OK;
+  if (!logits || !aligned16(logits) || !top_idx || (window > 0 && !history)) return RSWA_EINVAL;
+  return from_cuda(launch_ngram_topk(logits, ld, history, hist_ld, hist_len, rows, vocab, n,
+                                     window, k, mask_in_place, uniform,
+                                     uniform ? temperature : 1.f, top_idx, top_val, token,
+                                     device_error, (cudaStream_t)stream));
+}
+
 rswa_status rswa_get_ring(const rswa_state *s, int64_t *n_generated, int32_t *ring_pos,
                           int64_t *cache_len, void *stream) {
   if (!s) return RSWA_EINVAL;

@@ -1,0 +1,493 @@
+// Fused windowed n-gram ban + top-k selection over the vocabulary (greedy
+// decoding at k = 1, optional sampling among the k survivors).
+//
+// Method ("开源5天Star破万之后：百度Unlimited-OCR的爆火路径复盘", §2.3): inside
+// the sliding window of the generated history, every token that would repeat
+// an n-gram of size ngram_size gets score -inf; the next token is then chosen
+// from the masked scores.  Selection follows a total order: larger masked
+// value first, the lower column first among equal values; NaN ranks as -inf.
+//
+// Design (HBM-bound: each logit is read once):
+//  - One thread-block cluster of C = ceil(vocab / 16384) CTAs per row; each
+//    CTA holds its 16,384 columns in registers (64 per thread, 16 float4
+//    loads in flight per thread), so the row is read from HBM exactly once.
+//  - The ban: the row's history is staged in shared memory and every thread
+//    tests one candidate start of the windowed n-gram match at a time; the
+//    banned tokens in this CTA's columns are marked in a shared-memory
+//    bitmap (and, on request, -inf is stored over them in the logits).
+//  - Every column gets a 64-bit key: the order-preserving image of its masked
+//    value in the high word, (2^32 - 1 - column) in the low word, so keys
+//    are distinct and "larger key" is exactly the selection order.
+//  - k = 1 (its own kernel, nothing held): each thread streams its columns
+//    in increasing order keeping the first strict maximum, which costs one
+//    compare and two selects per column; the bitmap is consulted only when
+//    the maximum would change.  The (value, column) maxima are reduced over
+//    the warp, the CTA and, through distributed shared memory, the cluster.
+//    Few registers and little shared memory: the whole grid is one wave.
+//  - k > 1: radix select, 8 bits at a time from the top: each CTA histograms
+//    the digit of the keys that still match the chosen prefix, every CTA
+//    reads all CTAs' histograms through distributed shared memory and picks
+//    the digit holding the k-th largest key; this stops as soon as that
+//    digit's bin holds exactly the keys still needed (at the latest after
+//    the 8th digit, keys being distinct).  The keys at or above the final
+//    prefix -- exactly k -- go to the leader, which orders them.
+//  - Sampling: p_i proportional to exp((x_i - x_0) / T) over the k survivors
+//    (x_0 the largest), inverse CDF at the caller's uniform u in [0, 1).
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace rswa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kF4PerThread = 16;
+constexpr int kEPT = 4 * kF4PerThread;     // columns per thread
+constexpr int kChunk = kThreads * kEPT;    // columns per CTA
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxTopkCluster = 16;        // vocab <= 16 * kChunk
+static_assert(kTopkMax <= kThreads, "one thread per selected key");
+
+struct TopkSmem {
+  uint32_t ban_bits[kChunk / 32];
+  uint32_t hist[2][256];
+  uint32_t scan[kWarps];
+  unsigned long long cand[kTopkMax];       // leader: the selected keys
+  unsigned long long sorted[kTopkMax];
+  float prob[kTopkMax];
+  uint32_t n_cand;                          // leader: keys received
+  uint32_t sel_digit, sel_need, sel_done;  // radix decision of the pass
+};
+
+// Inverse of the order image (for the reported values).
+__device__ __forceinline__ float ord_value(uint32_t o) {
+  const uint32_t u = (o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o;
+  return __uint_as_float(u);
+}
+
+// Order-preserving image of a masked value, branch-free: NaN -> -inf via
+// fmaxf, -0 -> +0 via the addition, then the sign-dependent flip.
+__device__ __forceinline__ uint32_t ord_fast(float x) {
+  const float y = fmaxf(x, -INFINITY) + 0.0f;
+  const uint32_t u = __float_as_uint(y);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+}
+
+struct TopkArgs {
+  float *logits;
+  int64_t ld;
+  const int32_t *history;
+  int64_t hist_ld;
+  const int32_t *hist_len;
+  int rows, vocab, n, window, k, mask_in_place;
+  const float *uniform;
+  float inv_temp_log2e;  // log2(e) / T
+  int32_t *top_idx;
+  float *top_val;
+  int32_t *token;
+  int *err;
+};
+
+// Completes the staged history (hist_s, `window` ints), checks it, and marks the banned tokens that fall in [col0, col0 + kChunk)
+// in ban_bits (zeroed here), storing -inf over them when asked.  Returns the
+// row's error bits (the same in every CTA of the row).  Ends with a barrier.
+// Starts the copy of row `row`'s history (the first `window` tokens) into
+// shared memory; ban_prologue completes it.
+__device__ __forceinline__ void stage_history(const TopkArgs &a, int row, int32_t *hist_s) {
+  const int32_t *hist = a.history + (int64_t)row * a.hist_ld;
+  for (int i = threadIdx.x; i < a.window; i += kThreads) cp_async_4(hist_s + i, hist + i);
+}
+
+__device__ int ban_prologue(const TopkArgs &a, int row, int col0, uint32_t *ban_bits,
+                            int32_t *hist_s) {
+  const int tid = threadIdx.x;
+  const int h = a.hist_len ? __ldg(a.hist_len + row) : a.window;
+  const bool len_bad = h < 0 || h > a.window;
+  for (int i = tid; i < kChunk / 32; i += kThreads) ban_bits[i] = 0;
+  cp_async_wait_all();
+  __syncthreads();
+  bool tok_bad = false;
+  if (!len_bad)
+    for (int i = tid; i < h; i += kThreads) {
+      const int tok = hist_s[i];
+      tok_bad |= tok < 0 || tok >= a.vocab;
+    }
+  const int any_bad = __syncthreads_or(tok_bad);
+  if (len_bad) return RSWA_DEVERR_BAD_LENGTH;
+  if (any_bad) return RSWA_DEVERR_BAD_TOKEN;
+  if (h >= a.n) {
+    const int m = a.n - 1;
+    const int32_t *suffix = hist_s + (h - m);
+    float *lrow = a.logits + (int64_t)row * a.ld;
+    for (int i = tid; i + a.n <= h; i += kThreads) {
+      int j = 0;
+      while (j < m && hist_s[i + j] == suffix[j]) ++j;
+      if (j < m) continue;
+      const int f = hist_s[i + m] - col0;
+      if (f >= 0 && f < kChunk) {
+        atomicOr(&ban_bits[f >> 5], 1u << (f & 31));
+        if (a.mask_in_place) lrow[col0 + f] = -INFINITY;
+      }
+    }
+  }
+  __syncthreads();
+  return 0;
+}
+
+// Outputs of a rejected row (written by the leader CTA only).
+__device__ void reject_row(const TopkArgs &a, int row, int rank) {
+  if (rank != 0) return;
+  for (int i = threadIdx.x; i < a.k; i += kThreads) {
+    a.top_idx[(int64_t)row * a.k + i] = -1;
+    if (a.top_val) a.top_val[(int64_t)row * a.k + i] = __int_as_float(0x7fc00000);
+  }
+  if (threadIdx.x == 0 && a.token) a.token[row] = -1;
+}
+
+// k = 1: streaming per thread, no data held.  Each thread keeps the two
+// first maxima of its columns (the selection order restricted to them); the
+// ban is worked out while the last two batches of loads are in flight (the
+// history was copied asynchronously at the start).  If a thread's best is
+// banned its second is the answer, unless that is banned too, in which case
+// the thread rescans its columns (from L2) skipping banned ones -- which
+// needs two banned tokens among one thread's 64 columns.
+__global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs in one wave
+    ngram_top1_kernel(const TopkArgs a) {
+  __shared__ uint32_t ban_bits[kChunk / 32];
+  __shared__ unsigned long long warp_best[kWarps];
+  __shared__ unsigned long long cta_best[kMaxTopkCluster];
+  extern __shared__ int32_t hist_s[];
+  const int C = (int)(gridDim.x / (unsigned)a.rows);
+  const int row = (int)(blockIdx.x / (unsigned)C);
+  const int rank = (int)(blockIdx.x % (unsigned)C);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col0 = rank * kChunk;
+  const float *lrow = a.logits + (int64_t)row * a.ld;
+  // arrive now, wait before the first remote store: no CTA then writes into a
+  // peer that has not started, and the wait costs nothing by that time
+  cluster_arrive_relaxed();
+  stage_history(a, row, hist_s);
+
+  // two batches of 4 float4 in flight: load B0, B1; then consume one batch
+  // and load the next into its registers
+  constexpr int kBatch = 4;
+  static_assert(kF4PerThread == 4 * kBatch, "four batches per thread");
+  auto load_batch = [&](float4 *dst, int i0) {
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int c = col0 + 4 * (tid + kThreads * (i0 + i));
+      dst[i] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      // volatile: issued here, in this order, not sunk to the first use
+      if (c < a.vocab)
+        asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(dst[i].x), "=f"(dst[i].y), "=f"(dst[i].z), "=f"(dst[i].w)
+                     : "l"(lrow + c));
+    }
+  };
+  // columns in increasing order: strict comparisons keep the first of equals
+  const int first_col = col0 + 4 * tid;
+  float b1 = -INFINITY, b2 = -INFINITY;
+  int i1 = first_col, i2 = first_col;
+  auto consume = [&](const float4 *x, int i0) {
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int c = col0 + 4 * (tid + kThreads * (i0 + i));
+      const float e[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float v = c + u < a.vocab ? e[u] : -INFINITY;
+        const bool gt1 = v > b1, gt2 = v > b2;
+        b2 = gt1 ? b1 : (gt2 ? v : b2);
+        i2 = gt1 ? i1 : (gt2 ? c + u : i2);
+        b1 = gt1 ? v : b1;
+        i1 = gt1 ? c + u : i1;
+      }
+    }
+  };
+  float4 x0[kBatch], x1[kBatch];
+  load_batch(x0, 0);
+  load_batch(x1, kBatch);
+  consume(x0, 0);
+  load_batch(x0, 2 * kBatch);
+  consume(x1, kBatch);
+  load_batch(x1, 3 * kBatch);
+  const int bad = ban_prologue(a, row, col0, ban_bits, hist_s);
+  if (bad) {  // the same in every CTA of the row
+    if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
+    reject_row(a, row, rank);
+    cluster_wait_acquire();  // leave the start-of-kernel phase balanced
+    return;
+  }
+  consume(x0, 2 * kBatch);
+  consume(x1, 3 * kBatch);
+
+  const auto banned = [&](int col) {
+    const int f = col - col0;
+    return ((ban_bits[f >> 5] >> (f & 31)) & 1u) != 0;
+  };
+  float best = b1;
+  int bi = i1;
+  if (b1 != -INFINITY && banned(i1)) {
+    if (b2 == -INFINITY) {
+      best = -INFINITY;  // everything left ranks as -inf: the lowest column
+      bi = first_col;
+    } else if (!banned(i2)) {
+      best = b2;
+      bi = i2;
+    } else {
+      // rescan with the ban applied, 8 loads in flight at a time
+      best = -INFINITY;
+      bi = first_col;
+      for (int h0 = 0; h0 < kF4PerThread; h0 += 2 * kBatch) {
+        float4 y[2 * kBatch];
+#pragma unroll
+        for (int i = 0; i < 2 * kBatch; ++i) {
+          const int c = col0 + 4 * (tid + kThreads * (h0 + i));
+          y[i] = c < a.vocab ? *reinterpret_cast<const float4 *>(lrow + c)
+                             : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 2 * kBatch; ++i) {
+          const int c = col0 + 4 * (tid + kThreads * (h0 + i));
+          const float e[4] = {y[i].x, y[i].y, y[i].z, y[i].w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (c + u < a.vocab && e[u] > best && !banned(c + u)) {
+              best = e[u];
+              bi = c + u;
+            }
+        }
+      }
+    }
+  }
+  // (value, column) as one key: larger value first, then the lower column
+  unsigned long long key =
+      bi < a.vocab ? ((unsigned long long)ord_fast(best) << 32) | (0xFFFFFFFFu - (uint32_t)bi)
+                   : 0ull;
+#pragma unroll
+  for (int off = 16; off; off >>= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, off));
+  if (lane == 0) warp_best[warp] = key;
+  __syncthreads();
+  cluster_wait_acquire();  // every CTA of the cluster has started
+  if (tid == 0) {
+    unsigned long long b = 0;
+    for (int i = 0; i < kWarps; ++i) b = max(b, warp_best[i]);
+    st_cluster_u64(map_to_rank(&cta_best[rank], 0), b);  // into the leader
+  }
+  __syncwarp();
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (rank == 0 && tid == 0) {
+    unsigned long long b = 0;
+    for (int r = 0; r < C; ++r) b = max(b, cta_best[r]);
+    const int col = (int)(0xFFFFFFFFu - (uint32_t)b);
+    a.top_idx[row] = col;
+    if (a.top_val) a.top_val[row] = ord_value((uint32_t)(b >> 32));
+    if (a.token) a.token[row] = col;
+  }
+}
+
+// k > 1: the row's columns held in registers, radix select over the cluster.
+__global__ void __launch_bounds__(kThreads, 2)
+    ngram_topk_kernel(const TopkArgs a) {
+  __shared__ TopkSmem sm;
+  const int C = (int)(gridDim.x / (unsigned)a.rows);  // cluster size: CTAs per row
+  const int row = (int)(blockIdx.x / (unsigned)C);
+  const int rank = (int)(blockIdx.x % (unsigned)C);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col0 = rank * kChunk;
+  float *lrow = a.logits + (int64_t)row * a.ld;
+
+  // ---- issue this CTA's loads first (columns col0 + 4 * (tid + 256 i) + u)
+  float4 x[kF4PerThread];
+#pragma unroll
+  for (int i = 0; i < kF4PerThread; ++i) {
+    const int c = col0 + 4 * (tid + kThreads * i);
+    x[i] = c < a.vocab ? __ldcs(reinterpret_cast<const float4 *>(lrow + c))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  sm.hist[0][tid] = 0;
+  if (tid == 0) sm.n_cand = 0;
+  extern __shared__ int32_t hist_s[];
+  stage_history(a, row, hist_s);
+  const int bad = ban_prologue(a, row, col0, sm.ban_bits, hist_s);
+  if (bad) {  // the same in every CTA of the row: all leave before any cluster barrier
+    if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
+    reject_row(a, row, rank);
+    return;
+  }
+
+  // ---- keys: high word = order image of the masked value, low = ~column
+  uint32_t o[kEPT];
+#pragma unroll
+  for (int i = 0; i < kF4PerThread; ++i) {
+    const int c4 = 4 * (tid + kThreads * i);
+    const uint32_t bits = sm.ban_bits[c4 >> 5] >> (c4 & 31);
+    const float v[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool live = col0 + c4 + u < a.vocab;
+      o[4 * i + u] = !live ? 0u : ((bits >> u) & 1u) ? ord_fast(-INFINITY) : ord_fast(v[u]);
+    }
+  }
+  // low word of element e: 2^32 - 1 - column, an immediate offset from nb
+  const uint32_t nb = 0xFFFFFFFFu - (uint32_t)(col0 + 4 * tid);
+  auto key_of = [&](int e) -> unsigned long long {
+    const uint32_t lo = nb - (uint32_t)(4 * kThreads * (e >> 2) + (e & 3));
+    return ((unsigned long long)o[e] << 32) | (unsigned long long)lo;
+  };
+
+  cluster_arrive_relaxed();
+  cluster_wait_acquire();  // every CTA of the cluster has started
+
+  // ---- radix select, 8 bits per pass from the top of the 64-bit key
+  unsigned long long prefix = 0;  // chosen digits so far
+  uint32_t need = (uint32_t)a.k;
+  int pass = 0;
+  for (;; ++pass) {
+    const int buf = pass & 1;
+    const int shift = 56 - 8 * pass;  // this pass's digit
+#pragma unroll
+    for (int e = 0; e < kEPT; ++e) {
+      if (!o[e]) continue;
+      const unsigned long long key = key_of(e);
+      if (pass == 0 || (key >> (shift + 8)) == prefix)
+        atomicAdd(&sm.hist[buf][(uint32_t)(key >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    // bin (255 - tid) summed over the cluster; suffix sums = prefix scan of the reversed bins
+    const int bin = 255 - tid;
+    uint32_t cnt = 0;
+    for (int r = 0; r < C; ++r) cnt += ld_cluster_u32(map_to_rank(&sm.hist[buf][bin], r));
+    sm.hist[buf ^ 1][tid] = 0;  // the next pass's buffer (its readers are past this barrier)
+    uint32_t inc = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += y;
+    }
+    if (lane == 31) sm.scan[warp] = inc;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int i = 0; i < warp; ++i) before += sm.scan[i];
+    const uint32_t incl = before + inc;  // keys in bins >= bin
+    if (incl >= need && incl - cnt < need) {
+      sm.sel_digit = (uint32_t)bin;
+      sm.sel_need = need - (incl - cnt);
+      sm.sel_done = cnt == need - (incl - cnt);
+    }
+    __syncthreads();
+    prefix = (prefix << 8) | sm.sel_digit;
+    need = sm.sel_need;
+    if (sm.sel_done || pass == 7) break;
+  }
+  // ---- exactly k keys have their top (pass + 1) digits >= prefix
+  const int shift = 56 - 8 * pass;
+  const uint32_t cand_addr = map_to_rank(&sm.cand[0], 0);
+  const uint32_t count_addr = map_to_rank(&sm.n_cand, 0);
+#pragma unroll
+  for (int e = 0; e < kEPT; ++e) {
+    if (!o[e]) continue;
+    const unsigned long long key = key_of(e);
+    if ((key >> shift) >= prefix) {
+      const uint32_t slot = atom_add_cluster_u32(count_addr, 1u);
+      if (slot < (uint32_t)kTopkMax) st_cluster_u64(cand_addr + 8u * slot, key);
+    }
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (rank != 0) return;
+
+  // ---- leader: order the k keys, write them, sample
+  const int k = a.k;
+  if (tid < k) {
+    const unsigned long long mine = sm.cand[tid];
+    int r = 0;
+    for (int j = 0; j < k; ++j) r += sm.cand[j] > mine;
+    sm.sorted[r] = mine;
+  }
+  __syncthreads();
+  if (tid < k) {
+    const unsigned long long key = sm.sorted[tid];
+    const int col = (int)(0xFFFFFFFFu - (uint32_t)key);
+    const float val = ord_value((uint32_t)(key >> 32));
+    a.top_idx[(int64_t)row * k + tid] = col;
+    if (a.top_val) a.top_val[(int64_t)row * k + tid] = val;
+    const float x0 = ord_value((uint32_t)(sm.sorted[0] >> 32));
+    sm.prob[tid] = (val == -INFINITY || x0 == -INFINITY) ? 0.f
+                                                        : exp2f((val - x0) * a.inv_temp_log2e);
+  }
+  __syncthreads();
+  if (tid == 0 && a.token) {
+    int pick = 0;
+    if (a.uniform && sm.prob[0] > 0.f) {
+      float total = 0.f;
+      for (int i = 0; i < k; ++i) total += sm.prob[i];
+      const float target = a.uniform[row] * total;
+      float cum = 0.f;
+      pick = -1;
+      for (int i = 0; i < k; ++i) {
+        if (sm.prob[i] == 0.f) continue;
+        cum += sm.prob[i];
+        pick = i;
+        if (cum > target) break;
+      }
+    }
+    a.token[row] = (int)(0xFFFFFFFFu - (uint32_t)sm.sorted[pick]);
+  }
+}
+
+}  // namespace
+
+int topk_cluster_size(int vocab) { return (vocab + kChunk - 1) / kChunk; }
+
+cudaError_t launch_ngram_topk(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
+                              const int32_t *hist_len, int rows, int vocab, int n, int window,
+                              int k, int mask_in_place, const float *uniform, float temperature,
+                              int32_t *top_idx, float *top_val, int32_t *token, int *err,
+                              cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  const int C = topk_cluster_size(vocab);
+  void (*kernel)(TopkArgs) = k == 1 ? ngram_top1_kernel : ngram_topk_kernel;
+  if (C > 8) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  TopkArgs a;
+  a.logits = logits;
+  a.ld = ld;
+  a.history = history;
+  a.hist_ld = hist_ld;
+  a.hist_len = hist_len;
+  a.rows = rows;
+  a.vocab = vocab;
+  a.n = n;
+  a.window = window;
+  a.k = k;
+  a.mask_in_place = mask_in_place;
+  a.uniform = uniform;
+  a.inv_temp_log2e = 1.4426950408889634f / temperature;
+  a.top_idx = top_idx;
+  a.top_val = top_val;
+  a.token = token;
+  a.err = err;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)(rows * C));
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = (size_t)(window > 0 ? window : 1) * sizeof(int32_t);  // the history
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kernel, a);
+}
+
+}  // namespace rswa

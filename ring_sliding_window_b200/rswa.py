@@ -33,8 +33,9 @@ EXPORTED = (
     "rswa_decode_step_noalloc", "rswa_last_cuda_error", "rswa_debug_inject_fault",
     "rswa_decode_launch_shape", "rswa_pool_create", "rswa_pool_destroy", "rswa_pool_alloc",
     "rswa_pool_free", "rswa_pool_stats", "rswa_pool_capacity", "rswa_pool_cache_bytes",
-    "rswa_state_create_pooled",
+    "rswa_state_create_pooled", "rswa_ngram_topk",
 )
+RSWA_TOPK_MAX, RSWA_TOPK_MAX_VOCAB = 64, 262144
 RSWA_FAULT_DROP_DECODE_COPIES = 1
 RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
 
@@ -83,6 +84,9 @@ lib.rswa_ngram_mask.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, c
 lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
 lib.rswa_decode_launch_shape.argtypes = [_vp, _i32p, _i32p]
+lib.rswa_ngram_topk.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, ctypes.c_int32,
+                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                ctypes.c_int32, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
 lib.rswa_pool_create.argtypes = [ctypes.c_int64, ctypes.POINTER(_vp)]
 lib.rswa_pool_destroy.argtypes = [_vp]
 lib.rswa_pool_alloc.argtypes = [_vp, ctypes.c_int64, _i64p]
@@ -107,7 +111,7 @@ for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_deco
            "rswa_advance", "rswa_reset_ring", "rswa_ngram_mask", "rswa_get_ring",
            "rswa_check_device_error", "rswa_decode_launch_shape", "rswa_pool_create",
            "rswa_pool_destroy", "rswa_pool_alloc", "rswa_pool_free", "rswa_pool_stats",
-           "rswa_state_create_pooled"):
+           "rswa_state_create_pooled", "rswa_ngram_topk"):
     getattr(lib, _n).restype = ctypes.c_int
 
 
@@ -254,6 +258,30 @@ def rswa_ngram_mask(logits, history, hist_len, n: int, window: int, device_error
     _check(lib.rswa_ngram_mask(_ptr(logits), ld, _ptr(history), hist_ld, _ptr(hist_len), rows,
                                vocab, n, window, _ptr(device_error), _stream(stream)),
            "rswa_ngram_mask")
+
+
+def rswa_ngram_topk(logits, history, hist_len, n: int, window: int, k: int, mask_in_place=False,
+                    uniform=None, temperature: float = 1.0, top_idx=None, top_val=None,
+                    token=None, device_error=None, stream=None, vocab: Optional[int] = None):
+    """Fused n-gram ban + top-k (+ sampling).  logits: cuda float32 [rows, ld];
+    history: cuda int32 [rows, hist_ld].  Outputs are allocated when not given;
+    returns (top_idx [rows, k] int32, top_val [rows, k] float32, token [rows] int32)."""
+    rows = logits.shape[0]
+    ld = logits.stride(0) if rows else logits.shape[1]
+    vocab = logits.shape[1] if vocab is None else vocab
+    hist_ld = history.stride(0) if rows else window
+    dev = logits.device
+    if top_idx is None:
+        top_idx = torch.empty(rows, k, dtype=torch.int32, device=dev)
+    if top_val is None:
+        top_val = torch.empty(rows, k, dtype=torch.float32, device=dev)
+    if token is None:
+        token = torch.empty(rows, dtype=torch.int32, device=dev)
+    _check(lib.rswa_ngram_topk(_ptr(logits), ld, _ptr(history), hist_ld, _ptr(hist_len), rows,
+                               vocab, n, window, k, int(bool(mask_in_place)), _ptr(uniform),
+                               float(temperature), _ptr(top_idx), _ptr(top_val), _ptr(token),
+                               _ptr(device_error), _stream(stream)), "rswa_ngram_topk")
+    return top_idx, top_val, token
 
 
 def rswa_get_ring(state, batch: int, stream=None):

@@ -18,6 +18,10 @@ from ring_sliding_window_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
+def _bits(t):
+    return t.view(torch.int16 if t.element_size() == 2 else torch.int32)
+
+
 def _tol(dtype):
     return 2e-2 if dtype == torch.bfloat16 else 1e-5
 
@@ -44,7 +48,9 @@ def test_noalloc_matches_workspace_path_two_calls(dtype, d):
         torch.cuda.synchronize()
         diff = (got.double() - ref.double()).abs().max().item()
         assert diff <= _tol(dtype), (t, diff)
-        assert torch.equal(kc, st.k_cache[0]) and torch.equal(vc, st.v_cache[0]), t
+        # bit patterns: slots not yet written hold whatever the allocator left (maybe NaN)
+        assert torch.equal(_bits(kc), _bits(st.k_cache[0])), t
+        assert torch.equal(_bits(vc), _bits(st.v_cache[0])), t
     assert int(err.item()) == 0
     assert st.check() == 0
     st.close()
