@@ -179,7 +179,8 @@ def prefill_flops_per_layer(w: synth.Workload):
 class DecodeRig:
     """State, graph-captured token step and its I/O buffers for one workload."""
 
-    def __init__(self, w: synth.Workload, start_t: int, fill: str, stream: torch.cuda.Stream):
+    def __init__(self, w: synth.Workload, start_t: int, fill: str, stream: torch.cuda.Stream,
+                 rope: int = 0):
         from ring_sliding_window_b200 import rswa
         self.w, self.s = w, stream
         L, B, H, d = w.layers, w.batch, w.heads, w.head_dim
@@ -187,6 +188,8 @@ class DecodeRig:
         if w.n_generated is not None and fill != "prefill":
             ng = list(w.n_generated)
         self.st = rswa.State(B, L, H, d, w.window, w.prefill_lens, dtype=w.dtype, n_generated=ng)
+        if rope:
+            self.st.set_rope(rope, 10000.0, stream=stream)
         self.q = torch.empty(L, B, H, d, dtype=w.dtype, device="cuda")
         self.kn = torch.empty_like(self.q)
         self.vn = torch.empty_like(self.q)
@@ -478,6 +481,8 @@ def run_ours(args, rank, world, local_rank):
                 also.append(run_continuous_batching(args, s, hbm_peak))
             elif name == "ngram_topk":
                 also.append(run_ngram_topk(args, flush, s, hbm_peak))
+            elif name == "rope":
+                also.append(run_rope(args, flush, s, hbm_peak, tc_peak))
             else:
                 also.append(run_also(synth.workload(name), args, flush, s, hbm_peak, tc_peak))
             torch.cuda.empty_cache()
@@ -663,6 +668,40 @@ def run_ngram_topk(args, flush, s, hbm_peak, reps=5, calls=16, nbuf=4):
             "timing": f"CUDA graph of {calls} calls over {nbuf} logits buffers (> L2)", **out}
 
 
+def run_rope(args, flush, s, hbm_peak, tc_peak, steps=512):
+    """RoPE at cache-write time (absolute positions, theta = 10000) on the
+    single-page decode workload (the headline step with rotation on) and on
+    the multi-page prefill (2 layers; the rotation pre-pass is inside the
+    timed prefill).  The same measurements without RoPE sit beside them."""
+    w = synth.workload("single_page_decode")
+    res = {"workload": "rope (absolute positions, theta 10000)"}
+    for rope in (0, 1):
+        rig = DecodeRig(w, 0, "random", s, rope=rope)
+        rig.capture()
+        ms, _, _ = timed_tokens(rig, steps, args.warmup, flush)
+        launch_ms, t_at = timed_decode_launches(rig, 8, flush)
+        key = "rope" if rope else "no_rope"
+        res[f"single_page_{key}"] = {"decode_steps_per_s": steps / (sum(ms) / 1e3),
+                                     "avg_decode_launch_us": statistics.mean(launch_ms) * 1e3}
+        assert rig.st.check() == 0
+        rig.st.close()
+        del rig
+        torch.cuda.empty_cache()
+    wm = synth.workload("multi_page_decode")
+    w1 = synth.Workload(wm.name, wm.cfg_id, wm.dtype, wm.batch, 2, wm.heads, wm.head_dim,
+                        wm.window, wm.prefill_lens, 0)
+    for rope in (0, 1):
+        rig = DecodeRig(w1, 0, "prefill", s, rope=rope)
+        pf_ms = rig.prefill_all(flush)
+        f = prefill_flops_per_layer(w1) / (statistics.mean(pf_ms) / 1e3) / 1e12
+        res[f"multi_page_prefill_{'rope' if rope else 'no_rope'}"] = {
+            "tflops": f, "frac": f / tc_peak, "ms_per_layer": statistics.mean(pf_ms)}
+        rig.st.close()
+        del rig
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_also(w, args, flush, s, hbm_peak, tc_peak):
     steps = args.also_steps
     rig = DecodeRig(w, w.window, "random", s)
@@ -731,7 +770,7 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
     ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving,"
-                                      "continuous_batching,ngram_topk")
+                                      "continuous_batching,ngram_topk,rope")
     ap.add_argument("--also-steps", type=int, default=40)
     ap.add_argument("--skip-prefill-also", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

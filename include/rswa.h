@@ -36,8 +36,10 @@
  *    `device_error` word).  Nothing traps, aborts or waits without a bound.
  *  - Element types: RSWA_BF16 (bfloat16, round-to-nearest-even outputs with
  *    fp32 accumulation) or RSWA_F32.  head_dim is 64 or 128.
- *  - Heads: multi-head attention, num_kv_heads == num_heads.  Positions (RoPE)
- *    are the caller's business: keys are stored and used exactly as given.
+ *  - Heads: multi-head attention, num_kv_heads == num_heads.  Positions: by
+ *    default keys are stored and used exactly as given (the caller applies
+ *    any position encoding); rswa_state_set_rope moves the rotary embedding
+ *    into the library, applied when keys enter the cache.
  *
  * Layouts
  * -------
@@ -176,6 +178,39 @@ rswa_status rswa_state_create_pooled(const rswa_config *cfg, const int64_t *pref
                                      int64_t pool_slots, void *const *k_cache,
                                      void *const *v_cache, void *workspace, size_t workspace_size,
                                      void *stream, rswa_state **out);
+
+/* ------------------------------------------------------------------------
+ * Rotary position embedding at cache-write time.  The pages fix the cache
+ * (the prompt plus a ring of the W latest generated tokens; the model has
+ * max_position_embeddings = 32768, §2.1) but not the position a generated
+ * token takes once the ring has wrapped; the caller chooses:
+ *   RSWA_ROPE_ABSOLUTE : generated token t (0-based) of request b sits at
+ *                        position P_b + t -- the usual decoding positions;
+ *   RSWA_ROPE_SLOT     : it sits at the cache slot it is written to,
+ *                        P_b + (t mod W), so positions stay below P_b + W.
+ * Prompt token i is at position i under both.  The rotation is rotate-half
+ * (Llama family): for i < d/2 the pair (x_i, x_{i+d/2}) turns by the angle
+ * pos * theta^(-2i/d) (angles reduced in double precision, the rotation in
+ * float).  With RoPE on:
+ *  - rswa_prefill rotates k into the cache and q into `out` (used as
+ *    scratch: each query row is read there before its output overwrites it),
+ *    and attends with the rotated q and k; v is not rotated;
+ *  - rswa_decode_step rotates k_new before it enters the ring slot and q
+ *    before it is used, both at the token's position;
+ *  - the cache holds rotated keys (a resumed state's caller must have
+ *    rotated the keys it filled in the same way).
+ * ------------------------------------------------------------------------ */
+typedef enum rswa_rope_policy {
+  RSWA_ROPE_NONE = 0,
+  RSWA_ROPE_ABSOLUTE = 1,
+  RSWA_ROPE_SLOT = 2
+} rswa_rope_policy;
+
+/* Turn RoPE on (or off with RSWA_ROPE_NONE) for this state.  theta > 0 (the
+ * Llama default is 10000).  Call it before the state's first rswa_prefill or
+ * rswa_decode_step; it enqueues a small kernel on `stream`.  Returns
+ * RSWA_EINVAL for a bad policy or theta. */
+rswa_status rswa_state_set_rope(rswa_state *state, int32_t policy, float theta, void *stream);
 
 /* Free the host-side state.  Device memory stays the caller's. */
 rswa_status rswa_state_destroy(rswa_state *state);

@@ -203,6 +203,31 @@ def ngram_ban(logits: np.ndarray, history: np.ndarray, hist_len, n: int, window:
     return int(rc)
 
 
+def rope(x, pos, theta: float = 10000.0) -> np.ndarray:
+    """Rotary position embedding, rotate-half form, in FP64.
+
+    The pages give the model's max_position_embeddings (32768, §2.1) and name
+    Llama-style attention but define no position encoding; the reading here
+    is the Llama one: for i < d/2 the pair (x_i, x_{i+d/2}) turns by the angle
+    pos * theta^(-2i/d).  x: [n, ..., d]; pos: [n] positions of the n rows.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    inv_freq = float(theta) ** (-2.0 * np.arange(half, dtype=np.float64) / d)
+    ang = np.asarray(pos, dtype=np.float64).reshape((-1,) + (1,) * (x.ndim - 2) + (1,)) * inv_freq
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def rope_position(policy: str, prefill_len: int, t: int, window: int) -> int:
+    """Position of generated token t (0-based) of a request with prefill_len
+    prompt tokens: 'absolute' -> P + t; 'slot' -> the cache slot it is
+    written to, P + (t mod W) (the ring slot of the pages' §2.1)."""
+    return prefill_len + t if policy == "absolute" else prefill_len + t % window
+
+
 def ngram_topk(logits: np.ndarray, history: np.ndarray, hist_len, n: int, window: int, k: int):
     """Windowed n-gram ban, then the k best columns of the masked row.
 

@@ -77,6 +77,36 @@ struct __align__(128) DecodeSmem {
   uint64_t empty[S::kStages];
 };
 
+// Rotate this lane's slice of a row (rotate-half RoPE, pairs (i, i + D/2))
+// by the (cos, sin) table cs[D/2].  Lane li of a row's 8 lanes holds chunks
+// li + 8 j; when a lane holds at least two chunks the partner chunk is in the
+// same lane, otherwise (bf16, D = 64) it is in lane li ^ 4.
+template <typename T, int D>
+__device__ __forceinline__ void rope_lane(float *x, int li, const float2 *cs) {
+  using S = DecodeShape<T, D>;
+  constexpr int E = S::kElemPerChunk;
+  if constexpr (S::kChunksPerLane >= 2) {
+    constexpr int kHalf = S::kChunksPerLane / 2;
+#pragma unroll
+    for (int j = 0; j < kHalf; ++j)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float2 r = cs[(li + 8 * j) * E + e];
+        const float a0 = x[j * E + e], b0 = x[(j + kHalf) * E + e];
+        x[j * E + e] = a0 * r.x - b0 * r.y;
+        x[(j + kHalf) * E + e] = b0 * r.x + a0 * r.y;
+      }
+  } else {
+    const bool first = li < 4;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, x[e], 4);
+      const float2 r = cs[(li & 3) * E + e];
+      x[e] = first ? x[e] * r.x - other * r.y : x[e] * r.x + other * r.y;
+    }
+  }
+}
+
 struct DecodeArgs {
   DeviceView v;
   const void *q, *k_new, *v_new;
@@ -233,7 +263,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     const bool owner = wslot >= pc.key_begin && wslot < pc.key_end;
     const int64_t in_off = ((int64_t)pc.b * v.H + pc.h) * D;  // element offset into [B][H][D]
 
-    // q slice of this lane, pre-scaled into the log2 domain
+    // q slice of this lane (rotated at its position with RoPE on), pre-scaled
+    // into the log2 domain
     float qf[S::kEPL];
     {
       const uint8_t *qrow = (const uint8_t *)a.q + in_off * (int64_t)sizeof(T);
@@ -242,6 +273,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         const uint4 u = *reinterpret_cast<const uint4 *>(qrow + (li + 8 * j) * 16);
         Chunk<T>::widen(u, qf + j * S::kElemPerChunk);
       }
+      if (v.rope) rope_lane<T, D>(qf, li, v.rope_cs + (int64_t)pc.b * (D / 2));
       const float qs = v.scale * kLog2e;
 #pragma unroll
       for (int e = 0; e < S::kEPL; ++e) qf[e] *= qs;
@@ -254,12 +286,43 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
       const int64_t wrow = pc.row0 + wslot;
       uint8_t *kdst = (uint8_t *)a.kc + wrow * S::kRowBytes;
       uint8_t *vdst = (uint8_t *)a.vc + wrow * S::kRowBytes;
-      for (int c = tid; c < 2 * S::kChunks; c += 128) {
-        const bool isk = c < S::kChunks;
-        const int cc = isk ? c : c - S::kChunks;
-        const uint4 u = *reinterpret_cast<const uint4 *>((isk ? kn : vn) + cc * 16);
-        *reinterpret_cast<uint4 *>((isk ? sm.sub_k : sm.sub_v) + cc * 16) = u;
-        *reinterpret_cast<uint4 *>((isk ? kdst : vdst) + cc * 16) = u;
+      if (!v.rope) {
+        for (int c = tid; c < 2 * S::kChunks; c += 128) {
+          const bool isk = c < S::kChunks;
+          const int cc = isk ? c : c - S::kChunks;
+          const uint4 u = *reinterpret_cast<const uint4 *>((isk ? kn : vn) + cc * 16);
+          *reinterpret_cast<uint4 *>((isk ? sm.sub_k : sm.sub_v) + cc * 16) = u;
+          *reinterpret_cast<uint4 *>((isk ? kdst : vdst) + cc * 16) = u;
+        }
+      } else {
+        // k_new turns by its position before it enters the ring: chunk c and
+        // chunk c + kChunks/2 hold the pairs (i, i + d/2)
+        constexpr int kHalf = S::kChunks / 2;
+        const float2 *cs = v.rope_cs + (int64_t)pc.b * (D / 2);
+        for (int c = tid; c < kHalf + S::kChunks; c += 128) {
+          if (c < kHalf) {
+            float x[S::kElemPerChunk], y[S::kElemPerChunk];
+            Chunk<T>::widen(*reinterpret_cast<const uint4 *>(kn + c * 16), x);
+            Chunk<T>::widen(*reinterpret_cast<const uint4 *>(kn + (c + kHalf) * 16), y);
+#pragma unroll
+            for (int e = 0; e < S::kElemPerChunk; ++e) {
+              const float2 r = cs[c * S::kElemPerChunk + e];
+              const float a0 = x[e], b0 = y[e];
+              x[e] = a0 * r.x - b0 * r.y;
+              y[e] = b0 * r.x + a0 * r.y;
+            }
+            const uint4 ux = Chunk<T>::narrow(x), uy = Chunk<T>::narrow(y);
+            *reinterpret_cast<uint4 *>(sm.sub_k + c * 16) = ux;
+            *reinterpret_cast<uint4 *>(sm.sub_k + (c + kHalf) * 16) = uy;
+            *reinterpret_cast<uint4 *>(kdst + c * 16) = ux;
+            *reinterpret_cast<uint4 *>(kdst + (c + kHalf) * 16) = uy;
+          } else {
+            const int cc = c - kHalf;
+            const uint4 u = *reinterpret_cast<const uint4 *>(vn + cc * 16);
+            *reinterpret_cast<uint4 *>(sm.sub_v + cc * 16) = u;
+            *reinterpret_cast<uint4 *>(vdst + cc * 16) = u;
+          }
+        }
       }
       named_bar_sync(1, 128);
     }
@@ -548,6 +611,7 @@ cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
 }
 
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s) {
+  if (v.rope) return launch_advance_rope(v, s);
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3((v.B + 255) / 256);
   lc.blockDim = dim3(256);

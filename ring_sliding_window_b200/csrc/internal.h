@@ -32,7 +32,7 @@ struct WsLayout {
   size_t err;        // int32 device error word (+ int32 debug flags)
   size_t t;          // int64 [B]   tokens generated so far
   size_t plen;       // int32 [B]   P_b
-  size_t slot_base;  // int64 [B+1] sum_{b'<b} (P_b' + W)
+  size_t slot_base;  // int64 [B+1] first cache slot of each request
   size_t tok_base;   // int64 [B+1] sum_{b'<b} P_b'
   size_t tile_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kPrefillTile)
   size_t tile64_base;  // int32 [B+1] sum_{b'<b} ceil(P_b' / kSimtTile)
@@ -43,6 +43,7 @@ struct WsLayout {
   size_t bh_count;   // int32 [B*H]   pieces of (b, h) finished in this launch
   size_t part_ml;    // float2 [n_pieces] (running max in log2 units, sum)
   size_t part_o;     // float [n_pieces][d] unnormalised outputs
+  size_t rope_cs;    // float2 [B][d/2] (cos, sin) at each request's current position
   size_t total;
 };
 
@@ -85,6 +86,9 @@ struct DeviceView {
   int decode_grid;
   int n_pieces;
   int cluster_size;  // > 0: decode runs one ring per cluster of this many CTAs
+  int rope;          // rswa_rope_policy (0: keys and queries used as given)
+  float rope_theta;
+  float2 *rope_cs;   // [B][D/2] (cos, sin) of the position of each request's next token
   int64_t total_tokens;  // sum P_b
   int total_tiles;       // sum ceil(P_b / kPrefillTile)
   int total_tiles64;     // sum ceil(P_b / kSimtTile)
@@ -125,10 +129,19 @@ cudaError_t launch_ngram_topk(float *logits, int64_t ld, const int32_t *history,
                               cudaStream_t s);
 cudaError_t launch_cache_fill(const DeviceView &v, const void *k, const void *vv, void *kc,
                               void *vc, cudaStream_t s);
+// RoPE of the prompt: rotated k into cache slots [0, P_b), rotated q into `qr`.
+cudaError_t launch_rope_prefill(const DeviceView &v, const void *q, const void *k, void *qr,
+                                void *kc, cudaStream_t s);
+// (cos, sin) table of every request's next-token position (v.rope_cs).
+cudaError_t launch_rope_table(const DeviceView &v, cudaStream_t s);
+cudaError_t launch_advance_rope(const DeviceView &v, cudaStream_t s);
+// kc: NULL to read K from `k`; else K is read from this layer's cache
+// (rotated keys, RoPE), which holds kc_rows rows of d elements.
 cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,
-                                const void *vv, void *out, cudaStream_t s);
+                                const void *vv, void *out, const void *kc, cudaStream_t s);
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, const int4 *blocks, int n_blocks, cudaStream_t s);
+                              void *out, const int4 *blocks, int n_blocks, const void *kc,
+                              int64_t kc_rows, cudaStream_t s);
 
 // Prefill work list of the tensor-core kernel: blocks of two consecutive
 // 128-row query tiles of one (b, h), in launch order.

@@ -51,8 +51,8 @@ struct SimtShape {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(SimtShape<T, D>::kThreads)
-    prefill_simt_kernel(const DeviceView v, const T *__restrict__ q, const T *__restrict__ k,
-                        const T *__restrict__ vv, T *__restrict__ out) {
+    prefill_simt_kernel(const DeviceView v, const T *q, const T *__restrict__ k,
+                        const T *__restrict__ vv, T *out, const T *__restrict__ kc) {
   using S = SimtShape<T, D>;
   extern __shared__ __align__(16) float smem_f[];
   float *Ks = smem_f;                 // [kKeys][D]
@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(SimtShape<T, D>::kThreads)
   const int P = v.plen[b];
   const int64_t tok0 = v.tok_base[b];
   const int HD = v.H * D;
+  // K rows from the cache (rotated keys) when kc is given
+  const int64_t krow0 = (int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W);
 
   const int row = threadIdx.x / S::kTPR;
   const int sub = threadIdx.x % S::kTPR;
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(SimtShape<T, D>::kThreads)
       float kx = 0.f, vx = 0.f;
       if (kj < P) {
         const int64_t off = (tok0 + kj) * HD + h * D + e;
-        kx = to_float(k[off]);
+        kx = to_float(kc ? kc[(krow0 + kj) * D + e] : k[off]);
         vx = to_float(vv[off]);
       }
       Ks[idx] = kx;
@@ -184,7 +186,7 @@ __global__ void cache_fill_kernel(const DeviceView v, const uint8_t *__restrict_
 
 template <typename T, int D>
 cudaError_t launch_simt_t(const DeviceView &v, const void *q, const void *k, const void *vv,
-                          void *out, cudaStream_t s) {
+                          void *out, const void *kc, cudaStream_t s) {
   using S = SimtShape<T, D>;
   const int smem = 2 * S::kKeys * D * (int)sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(prefill_simt_kernel<T, D>,
@@ -192,20 +194,21 @@ cudaError_t launch_simt_t(const DeviceView &v, const void *q, const void *k, con
   if (e != cudaSuccess) return e;
   dim3 grid(v.total_tiles64, v.H);
   prefill_simt_kernel<T, D><<<grid, S::kThreads, smem, s>>>(v, (const T *)q, (const T *)k,
-                                                            (const T *)vv, (T *)out);
+                                                            (const T *)vv, (T *)out,
+                                                            (const T *)kc);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,
-                                const void *vv, void *out, cudaStream_t s) {
+                                const void *vv, void *out, const void *kc, cudaStream_t s) {
   if (v.total_tiles64 == 0) return cudaSuccess;
   if (v.dtype == RSWA_BF16)
-    return v.D == 128 ? launch_simt_t<__nv_bfloat16, 128>(v, q, k, vv, out, s)
-                      : launch_simt_t<__nv_bfloat16, 64>(v, q, k, vv, out, s);
-  return v.D == 128 ? launch_simt_t<float, 128>(v, q, k, vv, out, s)
-                    : launch_simt_t<float, 64>(v, q, k, vv, out, s);
+    return v.D == 128 ? launch_simt_t<__nv_bfloat16, 128>(v, q, k, vv, out, kc, s)
+                      : launch_simt_t<__nv_bfloat16, 64>(v, q, k, vv, out, kc, s);
+  return v.D == 128 ? launch_simt_t<float, 128>(v, q, k, vv, out, kc, s)
+                    : launch_simt_t<float, 64>(v, q, k, vv, out, kc, s);
 }
 
 cudaError_t launch_cache_fill(const DeviceView &v, const void *k, const void *vv, void *kc,

@@ -94,6 +94,7 @@ struct PrefillTcArgs {
   DeviceView v;
   const int4 *blocks;  // (b, h, first query tile, number of tiles 1|2)
   __nv_bfloat16 *out;
+  int k_from_cache;    // K tiles from the layer's cache (rotated keys) instead of k
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *err,
@@ -197,6 +198,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       int issued = 0;
+      // K from the cache: rows H * S_b + h * (P_b + W) + key of a [rows][128]
+      // map (rows past the prompt are ring slots: masked, like the causal
+      // overhang of the input layout)
+      const bool from_cache = is_k && a.k_from_cache;
+      const int x0 = from_cache ? 0 : xh;
+      const int y0 = from_cache ? (int)((int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W))
+                                : tok0;
       for (int j = 0; j < n_kv_all; ++j) {
         const int s = j % nst;
         uint64_t *empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
@@ -204,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *dst = is_k ? sm.k[s] : sm.v[s];
         if (!wait_bar(empty, ((j / nst) & 1) ^ 1, v.err, dead)) break;
         mbar_arrive_expect_tx(full, kTileBytes);
-        tc::tma_load_2d(dst, tm, xh, tok0 + j * kTile, full);
-        tc::tma_load_2d(dst + kHalfBytes, tm, xh + 64, tok0 + j * kTile, full);
+        tc::tma_load_2d(dst, tm, x0, y0 + j * kTile, full);
+        tc::tma_load_2d(dst + kHalfBytes, tm, x0 + 64, y0 + j * kTile, full);
         issued = j + 1;
       }
       // every load issued has landed before the CTA may exit (bounded)
@@ -439,18 +447,21 @@ bool make_tmap(CUtensorMap *m, const void *base, int64_t tokens, int H) {
 }  // namespace
 
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, const int4 *blocks, int n_blocks, cudaStream_t s) {
+                              void *out, const int4 *blocks, int n_blocks, const void *kc,
+                              int64_t kc_rows, cudaStream_t s) {
   if (n_blocks == 0) return cudaSuccess;
   if (v.D != kD || v.dtype != RSWA_BF16) return cudaErrorInvalidValue;
+  if (kc && (kc_rows < 1 || kc_rows >= (int64_t(1) << 31))) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, v.total_tokens, v.H) || !make_tmap(&tk, k, v.total_tokens, v.H) ||
-      !make_tmap(&tv, vv, v.total_tokens, v.H))
+  // the cache as [kc_rows][1 x 128]: the same encoding with H = 1
+  const bool k_ok = kc ? make_tmap(&tk, kc, kc_rows, 1) : make_tmap(&tk, k, v.total_tokens, v.H);
+  if (!make_tmap(&tq, q, v.total_tokens, v.H) || !k_ok || !make_tmap(&tv, vv, v.total_tokens, v.H))
     return cudaErrorInvalidValue;
   const int smem = (int)sizeof(PrefillSmem) + 1024;
   cudaError_t e =
       cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  PrefillTcArgs args{v, blocks, (__nv_bfloat16 *)out};
+  PrefillTcArgs args{v, blocks, (__nv_bfloat16 *)out, kc ? 1 : 0};
   prefill_tc_kernel<<<n_blocks, kThreads, smem, s>>>(tq, tk, tv, args);
   return cudaGetLastError();
 }

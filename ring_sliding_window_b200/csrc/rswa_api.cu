@@ -174,6 +174,7 @@ WsLayout layout_ws(const rswa_config *c, const int64_t *plen, const DecodePlan &
   w.bh_count = off;    off = align256(off + (B * c->num_heads) * sizeof(int32_t));
   w.part_ml = off;     off = align256(off + (size_t)p.n_pieces * sizeof(float2));
   w.part_o = off;      off = align256(off + (size_t)p.n_pieces * c->head_dim * sizeof(float));
+  w.rope_cs = off;     off = align256(off + B * (size_t)(c->head_dim / 2) * sizeof(float2));
   w.total = off;
   return w;
 }
@@ -376,6 +377,9 @@ rswa_status rswa_state_create_pooled(const rswa_config *cfg, const int64_t *pref
   v.decode_grid = s->plan.grid;
   v.n_pieces = s->plan.n_pieces;
   v.cluster_size = choose_cluster_size(cfg, prefill_len);
+  v.rope = RSWA_ROPE_NONE;
+  v.rope_theta = 10000.f;
+  v.rope_cs = (float2 *)(w + s->ws.rope_cs);
   v.total_tokens = tb[B];
   v.total_tiles = tl[B];
   v.total_tiles64 = tl64[B];
@@ -408,12 +412,20 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
     return RSWA_EINVAL;
   if (current_device() != s->device) return RSWA_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = launch_cache_fill(s->dv, k, v, s->k_cache[(size_t)layer], s->v_cache[(size_t)layer], st);
+  void *kc = s->k_cache[(size_t)layer];
+  cudaError_t e = launch_cache_fill(s->dv, k, v, kc, s->v_cache[(size_t)layer], st);
+  // RoPE: rotated k overwrites the cache's prompt slots, rotated q goes to
+  // `out`; attention then reads q from `out` and k from the cache
+  const bool rope = s->dv.rope != RSWA_ROPE_NONE;
+  if (e == cudaSuccess && rope) e = launch_rope_prefill(s->dv, q, k, out, kc, st);
+  const void *qa = rope ? (const void *)out : q;
+  const void *kca = rope ? (const void *)kc : nullptr;
   if (e == cudaSuccess) {
     if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128)
-      e = launch_prefill_tc(s->dv, q, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, st);
+      e = launch_prefill_tc(s->dv, qa, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, kca,
+                            (int64_t)s->cfg.num_heads * s->pool_slots, st);
     else
-      e = launch_prefill_simt(s->dv, q, k, v, out, st);
+      e = launch_prefill_simt(s->dv, qa, k, v, out, kca, st);
   }
   if (e != cudaSuccess) return from_cuda(e);
   s->layer_ready[(size_t)layer] = 1;
@@ -441,9 +453,11 @@ rswa_status rswa_advance(rswa_state *s, void *stream) {
 rswa_status rswa_reset_ring(rswa_state *s, void *stream) {
   if (!s) return RSWA_EINVAL;
   if (current_device() != s->device) return RSWA_EINVAL;
-  return from_cuda(cudaMemcpyAsync(s->dv.t, s->dv.t + s->cfg.batch,
-                                   (size_t)s->cfg.batch * sizeof(int64_t),
-                                   cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  cudaError_t e = cudaMemcpyAsync(s->dv.t, s->dv.t + s->cfg.batch,
+                                  (size_t)s->cfg.batch * sizeof(int64_t),
+                                  cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_rope_table(s->dv, (cudaStream_t)stream);
+  return from_cuda(e);
 }
 
 rswa_status rswa_ngram_mask(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
@@ -494,6 +508,17 @@ rswa_status rswa_get_ring(const rswa_state *s, int64_t *n_generated, int32_t *ri
     if (cache_len) cache_len[b] = s->plen[(size_t)b] + std::min(t[(size_t)b], W);
   }
   return RSWA_OK;
+}
+
+rswa_status rswa_state_set_rope(rswa_state *s, int32_t policy, float theta, void *stream) {
+  if (!s) return RSWA_EINVAL;
+  if (policy != RSWA_ROPE_NONE && policy != RSWA_ROPE_ABSOLUTE && policy != RSWA_ROPE_SLOT)
+    return RSWA_EINVAL;
+  if (!(theta > 0.f) || !isfinite(theta)) return RSWA_EINVAL;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  s->dv.rope = policy;
+  s->dv.rope_theta = theta;
+  return from_cuda(launch_rope_table(s->dv, (cudaStream_t)stream));
 }
 
 rswa_status rswa_decode_launch_shape(const rswa_state *s, int32_t *grid, int32_t *cluster_size) {
