@@ -483,6 +483,8 @@ def run_ours(args, rank, world, local_rank):
                 also.append(run_ngram_topk(args, flush, s, hbm_peak))
             elif name == "rope":
                 also.append(run_rope(args, flush, s, hbm_peak, tc_peak))
+            elif name == "standard_swa":
+                also.append(run_swa(args, flush, s, hbm_peak))
             else:
                 also.append(run_also(synth.workload(name), args, flush, s, hbm_peak, tc_peak))
             torch.cuda.empty_cache()
@@ -702,6 +704,49 @@ def run_rope(args, flush, s, hbm_peak, tc_peak, steps=512):
     return res
 
 
+def run_swa(args, flush, s, hbm_peak):
+    """Standard sliding-window contrast mode on the multi-page workload
+    (batch 8, prefill_len 8,256, W = 128): a decode step reads only the last
+    W positions of each ring; the prefill attends within the window.  Decode
+    per launch (steady state) and the 2-layer prefill, each beside the same
+    measurement in R-SWA mode."""
+    from ring_sliding_window_b200 import rswa
+    w = synth.workload("multi_page_decode")
+    res = {"workload": "standard_swa contrast (multi_page_decode shapes, W = 128)"}
+    row = w.heads * w.head_dim * w.elem_bytes
+    for mode in (rswa.RSWA_ATTN_RING, rswa.RSWA_ATTN_STANDARD_SWA):
+        rig = DecodeRig(w, w.window, "random", s)
+        rig.st.set_attention(mode)
+        rig.capture()
+        launch_ms, t_at = timed_decode_launches(rig, 8, flush)
+        us = statistics.mean(launch_ms) * 1e3
+        if mode == rswa.RSWA_ATTN_RING:
+            nbytes = kv_bytes_per_layer(w, t_at)
+        else:  # W keys per ring (t >= W - 1), plus q/k_new/v_new, ring write, out
+            nbytes = w.batch * (2 * w.window * row + 6 * row)
+        key = "ring" if mode == rswa.RSWA_ATTN_RING else "standard_swa"
+        res[f"decode_{key}"] = {"avg_launch_us": us, "algorithmic_bytes": nbytes,
+                                "gbs": nbytes / (us * 1e-6) / 1e9}
+        assert rig.st.check() == 0
+        rig.st.close()
+        del rig
+        torch.cuda.empty_cache()
+    w1 = synth.Workload(w.name, w.cfg_id, w.dtype, w.batch, 2, w.heads, w.head_dim, w.window,
+                        w.prefill_lens, 0)
+    rig = DecodeRig(w1, 0, "prefill", s)
+    rig.st.set_attention(rswa.RSWA_ATTN_STANDARD_SWA)
+    pf_ms = rig.prefill_all(flush)
+    flops = sum(4 * w.heads * w.head_dim * sum(min(i + 1, w.window) for i in range(P))
+                for P in w.prefill_lens)
+    res["prefill_standard_swa"] = {"ms_per_layer": statistics.mean(pf_ms),
+                                   "tflops": flops / (statistics.mean(pf_ms) / 1e3) / 1e12,
+                                   "kernel": "prefill_simt_kernel (CUDA cores)"}
+    rig.st.close()
+    del rig
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_also(w, args, flush, s, hbm_peak, tc_peak):
     steps = args.also_steps
     rig = DecodeRig(w, w.window, "random", s)
@@ -770,7 +815,7 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
     ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving,"
-                                      "continuous_batching,ngram_topk,rope")
+                                      "continuous_batching,ngram_topk,rope,standard_swa")
     ap.add_argument("--also-steps", type=int, default=40)
     ap.add_argument("--skip-prefill-also", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -212,6 +212,28 @@ typedef enum rswa_rope_policy {
  * RSWA_EINVAL for a bad policy or theta. */
 rswa_status rswa_state_set_rope(rswa_state *state, int32_t policy, float theta, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Standard sliding-window attention, the contrast the pages draw [§2.1: a
+ * standard sliding window would cut the prefill K/V as well, which for OCR
+ * loses image tokens; R-SWA keeps the whole prompt].  In this mode every
+ * token -- prompt and generated -- attends to the last W positions only,
+ * itself included: prompt query i to keys max(0, i - W + 1) .. i, and the
+ * t-th generated token (position P_b + t) to positions P_b + t - W + 1 ..
+ * P_b + t, i.e. the last W - 1 - t prompt tokens while t < W - 1 plus the
+ * ring.  The cache layout, the ring writes and rswa_advance are unchanged:
+ * the mode changes what is attended, not what is stored.  The prefill runs
+ * on the CUDA-core kernel; decode gives each ring a cluster of ceil(W / 64)
+ * CTAs.
+ * ------------------------------------------------------------------------ */
+typedef enum rswa_attention_mode {
+  RSWA_ATTN_RING = 0,          /* R-SWA (default) */
+  RSWA_ATTN_STANDARD_SWA = 1   /* the window also cuts the prompt */
+} rswa_attention_mode;
+
+/* Host only; takes effect for the calls enqueued after it.  RSWA_EINVAL for
+ * an unknown mode. */
+rswa_status rswa_state_set_attention(rswa_state *state, int32_t mode);
+
 /* Free the host-side state.  Device memory stays the caller's. */
 rswa_status rswa_state_destroy(rswa_state *state);
 

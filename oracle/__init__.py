@@ -203,6 +203,21 @@ def ngram_ban(logits: np.ndarray, history: np.ndarray, hist_len, n: int, window:
     return int(rc)
 
 
+def prefill_window(q, k, v, scale: float, window: int) -> np.ndarray:
+    """Standard sliding-window prefill, the contrast of "开源5天Star破万之后：
+    百度Unlimited-OCR的爆火路径复盘" §2.1 (a standard window would cut the
+    prompt's K/V too): query i of each head attends to keys
+    max(0, i - window + 1) .. i.  q, k, v: [P, H, d]; returns [P, H, d]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    P, H, d = q.shape
+    out = np.empty((P, H, d), dtype=np.float64)
+    for i in range(P):
+        lo = max(0, i - window + 1)
+        for h in range(H):
+            out[i, h] = attend(q[i, h], k[lo:i + 1, h], v[lo:i + 1, h], scale)
+    return out
+
+
 def rope(x, pos, theta: float = 10000.0) -> np.ndarray:
     """Rotary position embedding, rotate-half form, in FP64.
 

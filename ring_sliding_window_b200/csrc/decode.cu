@@ -107,6 +107,37 @@ __device__ __forceinline__ void rope_lane(float *x, int li, const float2 *cs) {
   }
 }
 
+// This step's key range of a piece, read after the grid-dependency wait:
+// [kb, ke) clipped to the cache entries held (P_b + min(t_b + 1, W)) and,
+// for the standard sliding window, to the slots of the last W positions,
+// [max(0, min(P_b, P_b + t_b - W + 1)), held).  A cluster CTA (rank of C)
+// re-splits that window evenly.  wslot: this step's ring slot, or -1 when
+// the piece lies wholly in the prompt (ring mode only).
+struct KeyRange {
+  int kb, ke, wslot;
+};
+__device__ __forceinline__ KeyRange resolve_range(const DeviceView &v, const DecodePiece &pc,
+                                                  int rank, int C) {
+  KeyRange r{pc.key_begin, pc.key_end, -1};
+  if (!v.swa && r.ke <= pc.plen) return r;  // no ring counter needed
+  const int64_t t = v.t[pc.b];
+  const int valid = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
+  r.wslot = pc.plen + (int)(t % v.W);
+  if (v.swa) {
+    const int64_t lo64 = (int64_t)pc.plen + t - v.W + 1;
+    const int lo = lo64 < 0 ? 0 : (lo64 > pc.plen ? pc.plen : (int)lo64);
+    if (C > 0) {
+      const int per = (valid - lo + C - 1) / C;
+      r.kb = min(lo + rank * per, valid);
+      r.ke = min(lo + (rank + 1) * per, valid);
+    } else {
+      r.kb = max(r.kb, lo);
+    }
+  }
+  r.ke = min(r.ke, valid);
+  return r;
+}
+
 struct DecodeArgs {
   DeviceView v;
   const void *q, *k_new, *v_new;
@@ -184,7 +215,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   // RSWA_DEVERR_TIMEOUT and the kernel still finishes.  The flag is written by
   // a host copy, which a kernel launched after it never overlaps.
   const bool drop_copies = (*v.fault & RSWA_FAULT_DROP_DECODE_COPIES) != 0;
-  if (warp == S::kConsumerWarps && lane == 0 && !drop_copies) {
+  // (The standard-sliding-window mode picks its keys from t_b: no prefetch.)
+  if (warp == S::kConsumerWarps && lane == 0 && !drop_copies && !v.swa) {
     const DecodePiece &pc = first_piece;
     const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
     const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
@@ -213,16 +245,11 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     bool dead = false;
     for (int p = p_begin; p < p_end && !dead; ++p) {
       const DecodePiece pc = p == p_begin ? first_piece : v.pieces[p];
-      // a piece wholly inside the prompt needs no ring counter
-      int ke = pc.key_end;
-      if (ke > pc.plen) {
-        const int64_t t = v.t[pc.b];
-        const int valid = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
-        ke = ke < valid ? ke : valid;
-      }
+      const KeyRange kr = resolve_range(v, pc, rank, kCluster ? v.cluster_size : 0);
+      const int ke = kr.ke;
       const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
       const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
-      const int k_first = pc.key_begin + (p == p_begin ? pre_stages * S::kStageRows : 0);
+      const int k_first = kr.kb + (p == p_begin ? pre_stages * S::kStageRows : 0);
       for (int k0 = k_first; k0 < ke; k0 += S::kStageRows) {
         const int rows = (ke - k0) < S::kStageRows ? (ke - k0) : S::kStageRows;
         if (!mbar_wait_bounded(&sm.empty[stage], (round & 1) ^ 1, v.err, RSWA_DEVERR_TIMEOUT)) {
@@ -252,15 +279,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
 
   for (int p = p_begin; p < p_end; ++p) {
     const DecodePiece pc = p == p_begin ? first_piece : v.pieces[p];
-    // ring position: only pieces reaching past the prompt need it
-    int ke = pc.key_end, wslot = -1;
-    if (ke > pc.plen) {
-      const int64_t t = v.t[pc.b];
-      const int valid = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
-      wslot = pc.plen + (int)(t % v.W);
-      ke = ke < valid ? ke : valid;
-    }
-    const bool owner = wslot >= pc.key_begin && wslot < pc.key_end;
+    const KeyRange kr = resolve_range(v, pc, rank, kCluster ? v.cluster_size : 0);
+    const int ke = kr.ke, wslot = kr.wslot;
+    const bool owner = wslot >= kr.kb && wslot < kr.ke;
     const int64_t in_off = ((int64_t)pc.b * v.H + pc.h) * D;  // element offset into [B][H][D]
 
     // q slice of this lane (rotated at its position with RoPE on), pre-scaled
@@ -332,7 +353,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
 #pragma unroll
     for (int e = 0; e < S::kEPL; ++e) o[e] = 0.f;
 
-    for (int k0 = pc.key_begin; k0 < ke; k0 += S::kStageRows) {
+    for (int k0 = kr.kb; k0 < ke; k0 += S::kStageRows) {
       const int rows = (ke - k0) < S::kStageRows ? (ke - k0) : S::kStageRows;
       if (!dead && !mbar_wait_bounded(&sm.full[stage], round & 1, v.err, RSWA_DEVERR_TIMEOUT))
         dead = true;

@@ -86,6 +86,7 @@ struct DeviceView {
   int decode_grid;
   int n_pieces;
   int cluster_size;  // > 0: decode runs one ring per cluster of this many CTAs
+  int swa;           // 1: standard sliding window (the window also cuts the prompt)
   int rope;          // rswa_rope_policy (0: keys and queries used as given)
   float rope_theta;
   float2 *rope_cs;   // [B][D/2] (cos, sin) of the position of each request's next token

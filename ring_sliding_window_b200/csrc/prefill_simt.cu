@@ -88,7 +88,9 @@ __global__ void __launch_bounds__(SimtShape<T, D>::kThreads)
   float m = -INFINITY, l = 0.f;
 
   const int last_key = min(qt * S::kRows + S::kRows, P);  // keys [0, last_key) may be needed
-  for (int k0 = 0; k0 < last_key; k0 += S::kKeys) {
+  // standard sliding window: query qi sees keys (qi - W, qi] only
+  const int first_key = v.swa ? max(0, qt * S::kRows - v.W + 1) / S::kKeys * S::kKeys : 0;
+  for (int k0 = first_key; k0 < last_key; k0 += S::kKeys) {
     __syncthreads();
     for (int idx = threadIdx.x; idx < S::kKeys * D; idx += S::kThreads) {
       const int r = idx / D, e = idx % D;
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(SimtShape<T, D>::kThreads)
 #pragma unroll
         for (int x = 1; x < S::kTPR; x <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, x);
         const int kpos = k0 + kr;
-        sc[jj] = (row_ok && kr < kend && kpos <= qi) ? acc : -INFINITY;
+        sc[jj] = (row_ok && kr < kend && kpos <= qi && (!v.swa || kpos > qi - v.W)) ? acc
+                                                                                    : -INFINITY;
       }
       float m_new = m;
 #pragma unroll

@@ -30,37 +30,60 @@ __device__ __forceinline__ float2 rope_cs(int64_t pos, int i, int d, float theta
   return make_float2((float)cs, (float)sn);
 }
 
-// One thread per (prompt token, pair i): the angle is computed once and
-// applied to q and k of every head.
+// One CTA per run of kRun consecutive prompt positions of one sequence.
+// Thread i < d/2 reduces the run's first angle for pair i once (double
+// sincos) and walks the run with the angle-addition recurrence in double
+// precision (kRun steps add a few 1e-16), leaving float (cos, sin) in shared
+// memory; then all threads rotate q and k of every head of the run, with
+// consecutive threads on consecutive elements.
+constexpr int kRun = 64;
+
 template <typename T>
-__global__ void rope_prefill_kernel(const DeviceView v, const T *__restrict__ q,
-                                    const T *__restrict__ k, T *__restrict__ qr,
-                                    T *__restrict__ kc) {
+__global__ void __launch_bounds__(256)
+    rope_prefill_kernel(const DeviceView v, const T *__restrict__ q, const T *__restrict__ k,
+                        T *__restrict__ qr, T *__restrict__ kc) {
+  __shared__ float2 cs[kRun][64];
   const int half = v.D / 2;
-  const int64_t total = v.total_tokens * half;
-  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
-       w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t tk = w / half;
-    const int i = (int)(w % half);
-    int lo = 0, hi = v.B;  // sequence of token tk: tok_base[lo] <= tk < tok_base[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (v.tok_base[mid] <= tk) lo = mid; else hi = mid;
+  const int run = blockIdx.x;
+  int lo = 0, hi = v.B;  // sequence of the run: tile64_base[lo] <= run < tile64_base[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (v.tile64_base[mid] <= run) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int P = v.plen[b];
+  const int p0 = (run - v.tile64_base[b]) * kRun;
+  const int n = min(kRun, P - p0);
+  const int i = threadIdx.x;
+  if (i < half) {
+    const double inv_freq = pow((double)v.rope_theta, -2.0 * (double)i / (double)v.D);
+    double sn, c, sd, cd;
+    sincos((double)p0 * inv_freq, &sn, &c);
+    sincos(inv_freq, &sd, &cd);
+    for (int j = 0; j < n; ++j) {
+      cs[j][i] = make_float2((float)c, (float)sn);
+      const double cn = c * cd - sn * sd;  // angle + inv_freq
+      sn = sn * cd + c * sd;
+      c = cn;
     }
-    const int b = lo;
-    const int64_t slot = tk - v.tok_base[b];  // = the prompt position
-    const int P = v.plen[b];
-    const float2 cs = rope_cs(slot, i, v.D, v.rope_theta);
-    for (int h = 0; h < v.H; ++h) {
-      const int64_t src = (tk * v.H + h) * v.D;
-      const int64_t drow = ((int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W) + slot) * v.D;
-      const float qa = to_float(q[src + i]), qb = to_float(q[src + i + half]);
-      const float ka = to_float(k[src + i]), kb = to_float(k[src + i + half]);
-      qr[src + i] = from_float<T>(qa * cs.x - qb * cs.y);
-      qr[src + i + half] = from_float<T>(qb * cs.x + qa * cs.y);
-      kc[drow + i] = from_float<T>(ka * cs.x - kb * cs.y);
-      kc[drow + i + half] = from_float<T>(kb * cs.x + ka * cs.y);
-    }
+  }
+  __syncthreads();
+  const int per_pos = v.H * half;
+  const int64_t tok0 = v.tok_base[b] + p0;
+  const int64_t krow0 = (int64_t)v.H * v.slot_base[b] + p0;
+  for (int e = threadIdx.x; e < n * per_pos; e += blockDim.x) {
+    const int j = e / per_pos;
+    const int rem = e - j * per_pos;
+    const int h = rem / half, ii = rem - h * half;
+    const float2 r = cs[j][ii];
+    const int64_t src = ((tok0 + j) * v.H + h) * v.D + ii;
+    const int64_t dst = (krow0 + (int64_t)h * (P + v.W) + j) * v.D + ii;
+    const float qa = to_float(q[src]), qb = to_float(q[src + half]);
+    const float ka = to_float(k[src]), kb = to_float(k[src + half]);
+    qr[src] = from_float<T>(qa * r.x - qb * r.y);
+    qr[src + half] = from_float<T>(qb * r.x + qa * r.y);
+    kc[dst] = from_float<T>(ka * r.x - kb * r.y);
+    kc[dst + half] = from_float<T>(kb * r.x + ka * r.y);
   }
 }
 
@@ -90,29 +113,20 @@ __global__ void advance_rope_kernel(const DeviceView v) {
     v.rope_cs[(int64_t)b * half + i] = rope_cs(pos, i, v.D, v.rope_theta);
 }
 
-int grid_for(int64_t work, int threads) {
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t blocks = (work + threads - 1) / threads;
-  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-  return (int)(blocks < 1 ? 1 : blocks);
-}
-
 }  // namespace
 
 cudaError_t launch_rope_prefill(const DeviceView &v, const void *q, const void *k, void *qr,
                                 void *kc, cudaStream_t s) {
   if (v.total_tokens == 0) return cudaSuccess;
-  const int threads = 256;
-  const int grid = grid_for(v.total_tokens * (v.D / 2), threads);
+  static_assert(kRun == kSimtTile, "runs are counted by the 64-token tile table");
+  const int grid = v.total_tiles64;
   if (v.dtype == RSWA_BF16)
-    rope_prefill_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(
+    rope_prefill_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
         v, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (__nv_bfloat16 *)qr,
         (__nv_bfloat16 *)kc);
   else
-    rope_prefill_kernel<float><<<grid, threads, 0, s>>>(v, (const float *)q, (const float *)k,
-                                                         (float *)qr, (float *)kc);
+    rope_prefill_kernel<float><<<grid, 256, 0, s>>>(v, (const float *)q, (const float *)k,
+                                                    (float *)qr, (float *)kc);
   return cudaGetLastError();
 }
 

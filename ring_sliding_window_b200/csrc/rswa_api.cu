@@ -377,6 +377,7 @@ rswa_status rswa_state_create_pooled(const rswa_config *cfg, const int64_t *pref
   v.decode_grid = s->plan.grid;
   v.n_pieces = s->plan.n_pieces;
   v.cluster_size = choose_cluster_size(cfg, prefill_len);
+  v.swa = 0;
   v.rope = RSWA_ROPE_NONE;
   v.rope_theta = 10000.f;
   v.rope_cs = (float2 *)(w + s->ws.rope_cs);
@@ -421,7 +422,9 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
   const void *qa = rope ? (const void *)out : q;
   const void *kca = rope ? (const void *)kc : nullptr;
   if (e == cudaSuccess) {
-    if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128)
+    // the standard sliding window runs on the CUDA-core kernel (its work,
+    // W keys per query, is too small for the tensor-core pipeline)
+    if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128 && !s->dv.swa)
       e = launch_prefill_tc(s->dv, qa, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, kca,
                             (int64_t)s->cfg.num_heads * s->pool_slots, st);
     else
@@ -519,6 +522,21 @@ rswa_status rswa_state_set_rope(rswa_state *s, int32_t policy, float theta, void
   s->dv.rope = policy;
   s->dv.rope_theta = theta;
   return from_cuda(launch_rope_table(s->dv, (cudaStream_t)stream));
+}
+
+rswa_status rswa_state_set_attention(rswa_state *s, int32_t mode) {
+  if (!s) return RSWA_EINVAL;
+  if (mode != RSWA_ATTN_RING && mode != RSWA_ATTN_STANDARD_SWA) return RSWA_EINVAL;
+  s->dv.swa = mode == RSWA_ATTN_STANDARD_SWA;
+  // the window holds at most W keys per ring: one cluster of ceil(W / 64)
+  // CTAs per ring (clusters are independent, so any batch size runs)
+  const char *env = getenv("RSWA_DECODE_SPLIT");
+  const bool force_streamk = env && strcmp(env, "streamk") == 0;
+  if (s->dv.swa && !force_streamk)
+    s->dv.cluster_size = std::max(1, std::min(16, (s->cfg.window + 63) / 64));
+  else
+    s->dv.cluster_size = choose_cluster_size(&s->cfg, s->plen.data());
+  return RSWA_OK;
 }
 
 rswa_status rswa_decode_launch_shape(const rswa_state *s, int32_t *grid, int32_t *cluster_size) {

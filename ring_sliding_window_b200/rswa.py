@@ -34,7 +34,9 @@ EXPORTED = (
     "rswa_decode_launch_shape", "rswa_pool_create", "rswa_pool_destroy", "rswa_pool_alloc",
     "rswa_pool_free", "rswa_pool_stats", "rswa_pool_capacity", "rswa_pool_cache_bytes",
     "rswa_state_create_pooled", "rswa_ngram_topk", "rswa_state_set_rope",
+    "rswa_state_set_attention",
 )
+RSWA_ATTN_RING, RSWA_ATTN_STANDARD_SWA = 0, 1
 RSWA_ROPE_NONE, RSWA_ROPE_ABSOLUTE, RSWA_ROPE_SLOT = 0, 1, 2
 RSWA_TOPK_MAX, RSWA_TOPK_MAX_VOCAB = 64, 262144
 RSWA_FAULT_DROP_DECODE_COPIES = 1
@@ -86,6 +88,7 @@ lib.rswa_get_ring.argtypes = [_vp, _i64p, _i32p, _i64p, _vp]
 lib.rswa_check_device_error.argtypes = [_vp, _vp]
 lib.rswa_decode_launch_shape.argtypes = [_vp, _i32p, _i32p]
 lib.rswa_state_set_rope.argtypes = [_vp, ctypes.c_int32, ctypes.c_float, _vp]
+lib.rswa_state_set_attention.argtypes = [_vp, ctypes.c_int32]
 lib.rswa_ngram_topk.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, ctypes.c_int32,
                                 ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                 ctypes.c_int32, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
@@ -113,7 +116,8 @@ for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_deco
            "rswa_advance", "rswa_reset_ring", "rswa_ngram_mask", "rswa_get_ring",
            "rswa_check_device_error", "rswa_decode_launch_shape", "rswa_pool_create",
            "rswa_pool_destroy", "rswa_pool_alloc", "rswa_pool_free", "rswa_pool_stats",
-           "rswa_state_create_pooled", "rswa_ngram_topk", "rswa_state_set_rope"):
+           "rswa_state_create_pooled", "rswa_ngram_topk", "rswa_state_set_rope",
+           "rswa_state_set_attention"):
     getattr(lib, _n).restype = ctypes.c_int
 
 
@@ -300,6 +304,10 @@ def rswa_state_set_rope(state, policy: int, theta: float = 10000.0, stream=None)
            "rswa_state_set_rope")
 
 
+def rswa_state_set_attention(state, mode: int) -> None:
+    _check(lib.rswa_state_set_attention(state, int(mode)), "rswa_state_set_attention")
+
+
 def rswa_decode_launch_shape(state):
     """(grid, cluster_size) of this state's decode launches; cluster_size 0 = stream-K split."""
     g, c = ctypes.c_int32(0), ctypes.c_int32(0)
@@ -402,6 +410,9 @@ class State:
 
     def set_rope(self, policy: int, theta: float = 10000.0, stream=None):
         rswa_state_set_rope(self.handle, policy, theta, stream)
+
+    def set_attention(self, mode: int):
+        rswa_state_set_attention(self.handle, mode)
 
 
 class TokenPool:

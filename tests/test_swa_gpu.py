@@ -1,0 +1,84 @@
+"""Standard sliding-window mode (rswa_state_set_attention) against the FP64
+oracle: the contrast the pages draw in "开源5天Star破万之后：百度Unlimited-OCR
+的爆火路径复盘" §2.1 -- a standard window also cuts the prompt.
+
+Prompt query i attends to keys (i - W, i]; generated token t (position
+P + t) to positions (P + t - W, P + t], taken here by brute force from the
+token history (not from any cache).  The ring writes are the same as in
+R-SWA mode, so the caches still match the ring oracle bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import f64, seq_slices, tol_for
+from ring_sliding_window_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("split", ["auto", "streamk"])
+@pytest.mark.parametrize("W", [8, 130])
+def test_standard_swa_prefill_and_decode(dtype, d, split, W, monkeypatch):
+    from ring_sliding_window_b200 import rswa
+    if split != "auto":
+        monkeypatch.setenv("RSWA_DECODE_SPLIT", split)
+    B, L, H, P, steps = 2, 2, 2, (200, 37), 20 if W == 8 else 140
+    w = synth.Workload("swa", 71 + W, dtype, B, L, H, d, W, P, steps)
+    st = rswa.State(B, L, H, d, W, P, dtype=dtype)
+    st.set_attention(rswa.RSWA_ATTN_STANDARD_SWA)
+    grid, csize = st.decode_launch_shape()
+    assert (csize == 0) == (split == "streamk")
+    tol = tol_for(dtype)
+    sl = seq_slices(P)
+    model = oracle.RingModel(P, W, L, H, d)
+    hist_k = [[None] * B for _ in range(L)]
+    hist_v = [[None] * B for _ in range(L)]
+    for l in range(L):
+        q, k, v = synth.prefill_qkv(w, l, "cuda")
+        out = torch.empty_like(q)
+        st.prefill(l, q, k, v, out)
+        for b in range(B):
+            ref = oracle.prefill_window(f64(q[sl[b]]), f64(k[sl[b]]), f64(v[sl[b]]), w.scale, W)
+            assert np.max(np.abs(f64(out[sl[b]]) - ref)) <= tol, (l, b)
+            hist_k[l][b], hist_v[l][b] = list(f64(k[sl[b]])), list(f64(v[sl[b]]))
+            model.prefill(l, b, f64(k[sl[b]]), f64(v[sl[b]]))
+    for t in range(steps):
+        for l in range(L):
+            q, kn, vn = synth.decode_qkv(w, l, t, "cuda")
+            out = torch.empty_like(q)
+            st.decode_step(l, q, kn, vn, out)
+            for b in range(B):
+                model.rings[l][b].step(f64(q[b]), f64(kn[b]), f64(vn[b]), w.scale)
+                hist_k[l][b].append(f64(kn[b]))
+                hist_v[l][b].append(f64(vn[b]))
+                K = np.stack(hist_k[l][b][-W:])  # the last W positions, this token included
+                V = np.stack(hist_v[l][b][-W:])
+                for h in range(H):
+                    ref = oracle.attend(f64(q[b, h]), K[:, h], V[:, h], w.scale)
+                    err = np.max(np.abs(f64(out[b, h]) - ref))
+                    assert err <= tol, (t, l, b, h, err)
+        st.advance()
+    for l in range(L):
+        for b in range(B):
+            kc, vc, held = model.rings[l][b].snapshot()
+            for h in range(H):
+                assert np.array_equal(f64(st.cache_view(l, "k", b, h)[:held]), kc[:held, h])
+                assert np.array_equal(f64(st.cache_view(l, "v", b, h)[:held]), vc[:held, h])
+    assert st.check() == 0
+
+
+def test_attention_mode_switch_and_errors():
+    from ring_sliding_window_b200 import rswa
+    st = rswa.State(1, 1, 2, 128, 8, [64], dtype=torch.bfloat16)
+    for bad in (2, -1):
+        with pytest.raises(rswa.RswaError) as e:
+            st.set_attention(bad)
+        assert e.value.status == rswa.RSWA_EINVAL
+    ring_shape = st.decode_launch_shape()
+    st.set_attention(rswa.RSWA_ATTN_STANDARD_SWA)
+    assert st.decode_launch_shape()[1] == 1  # ceil(8 / 64) CTAs per ring
+    st.set_attention(rswa.RSWA_ATTN_RING)
+    assert st.decode_launch_shape() == ring_shape
