@@ -59,6 +59,16 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define RSWA_EXP2_FMA_EVERY 0
 #endif
 constexpr int kEmuEvery = RSWA_EXP2_FMA_EVERY;
+// 1: P's exponentials in packed bf16 pairs (ex2.approx.ftz.bf16x2): the
+// argument x = s * scale*log2(e) - m is rounded to bf16 first (8-bit
+// mantissa), the result is the bf16 P the P V product reads anyway, and the
+// row sum adds the same rounded values.  Half the MUFU operations of the
+// fp32 path, but measured slower on B200 (804 vs 858 TFLOP/s multi-page),
+// so off by default.  Build-time knob: -DRSWA_EXP2_BF16X2=0|1.
+#ifndef RSWA_EXP2_BF16X2
+#define RSWA_EXP2_BF16X2 0
+#endif
+constexpr bool kExpBf16x2 = RSWA_EXP2_BF16X2 != 0;
 // 1: the two softmax warpgroups take turns on their exponential loops
 // (A(0), B(0), A(1), B(1), ...), keeping them half a period apart so each
 // has the MUFU pipe to itself while the tensor core runs the other tile's
@@ -338,12 +348,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t xx = tc::ffma2(tc::f2_pack(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]),
                                         sl2x2, negm2);
           const float x0 = tc::f2_lo(xx), x1 = tc::f2_hi(xx);
-          // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
-          const bool emu = kEmuEvery > 0 && (c % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
-          const float p0 = emu ? tc::exp2_fma(x0) : tc::ex2(x0);
-          const float p1 = emu ? tc::exp2_fma(x1) : tc::ex2(x1);
-          rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(p0, p1));
-          pk[c] = tc::pack_bf16x2(p0, p1);
+          if constexpr (kExpBf16x2) {
+            // both exponentials in one MUFU op, straight into the bf16 pair
+            // that P V consumes; the row sum adds exactly those values
+            const uint32_t pb = tc::ex2_bf16x2(tc::pack_bf16x2(x0, x1));
+            rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(__uint_as_float(pb << 16),
+                                                            __uint_as_float(pb & 0xffff0000u)));
+            pk[c] = pb;
+          } else {
+            // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
+            const bool emu =
+                kEmuEvery > 0 && (c % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
+            const float p0 = emu ? tc::exp2_fma(x0) : tc::ex2(x0);
+            const float p1 = emu ? tc::exp2_fma(x1) : tc::ex2(x1);
+            rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(p0, p1));
+            pk[c] = tc::pack_bf16x2(p0, p1);
+          }
         }
         tc::st32(t_s + 32 * half, pk);
       }

@@ -48,18 +48,12 @@ constexpr int kEPT = 4 * kF4PerThread;     // columns per thread
 constexpr int kChunk = kThreads * kEPT;    // columns per CTA
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTopkCluster = 16;        // vocab <= 16 * kChunk
+// leader's candidate buffer: the C x 256 thread maxima first, then the keys
+// >= T (at most 64 per thread of the k threads whose maximum is >= T)
+constexpr int kTopkCandidates = 64 * kTopkMax;
+static_assert(kMaxTopkCluster * kThreads <= kTopkCandidates, "thread maxima fit the buffer");
 static_assert(kTopkMax <= kThreads, "one thread per selected key");
 
-struct TopkSmem {
-  uint32_t ban_bits[kChunk / 32];
-  uint32_t hist[2][256];
-  uint32_t scan[kWarps];
-  unsigned long long cand[kTopkMax];       // leader: the selected keys
-  unsigned long long sorted[kTopkMax];
-  float prob[kTopkMax];
-  uint32_t n_cand;                          // leader: keys received
-  uint32_t sel_digit, sel_need, sel_done;  // radix decision of the pass
-};
 
 // Inverse of the order image (for the reported values).
 __device__ __forceinline__ float ord_value(uint32_t o) {
@@ -146,32 +140,23 @@ __device__ void reject_row(const TopkArgs &a, int row, int rank) {
   if (threadIdx.x == 0 && a.token) a.token[row] = -1;
 }
 
-// k = 1: streaming per thread, no data held.  Each thread keeps the two
-// first maxima of its columns (the selection order restricted to them); the
-// ban is worked out while the last two batches of loads are in flight (the
-// history was copied asynchronously at the start).  If a thread's best is
-// banned its second is the answer, unless that is banned too, in which case
-// the thread rescans its columns (from L2) skipping banned ones -- which
-// needs two banned tokens among one thread's 64 columns.
-__global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs in one wave
-    ngram_top1_kernel(const TopkArgs a) {
-  __shared__ uint32_t ban_bits[kChunk / 32];
-  __shared__ unsigned long long warp_best[kWarps];
-  __shared__ unsigned long long cta_best[kMaxTopkCluster];
-  extern __shared__ int32_t hist_s[];
-  const int C = (int)(gridDim.x / (unsigned)a.rows);
-  const int row = (int)(blockIdx.x / (unsigned)C);
-  const int rank = (int)(blockIdx.x % (unsigned)C);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int col0 = rank * kChunk;
+// The streaming pass shared by both kernels: each thread reads its 64 columns
+// once (two batches of four 16-byte loads in flight) and keeps the two first
+// maxima of them in increasing column order; the ban is worked out while the
+// last two batches are in flight (the history was copied asynchronously at
+// the start).  If a thread's best is banned its second is the answer, unless
+// that is banned too, in which case the thread rescans its columns (from L2)
+// skipping banned ones -- which needs two banned tokens among one thread's 64
+// columns.  Returns the thread's largest masked key ((order image of the
+// masked value) << 32 | ~column), 0 if it has no column, and sets *bad to
+// the row's error bits (the same in every CTA of the row).
+template <bool kEvictFirst>
+__device__ __forceinline__ unsigned long long stream_thread_max(const TopkArgs &a, int row,
+                                                                int col0, uint32_t *ban_bits,
+                                                                int32_t *hist_s, int *bad) {
+  const int tid = threadIdx.x;
   const float *lrow = a.logits + (int64_t)row * a.ld;
-  // arrive now, wait before the first remote store: no CTA then writes into a
-  // peer that has not started, and the wait costs nothing by that time
-  cluster_arrive_relaxed();
   stage_history(a, row, hist_s);
-
-  // two batches of 4 float4 in flight: load B0, B1; then consume one batch
-  // and load the next into its registers
   constexpr int kBatch = 4;
   static_assert(kF4PerThread == 4 * kBatch, "four batches per thread");
   auto load_batch = [&](float4 *dst, int i0) {
@@ -180,10 +165,16 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
       const int c = col0 + 4 * (tid + kThreads * (i0 + i));
       dst[i] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
       // volatile: issued here, in this order, not sunk to the first use
-      if (c < a.vocab)
-        asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
-                     : "=f"(dst[i].x), "=f"(dst[i].y), "=f"(dst[i].z), "=f"(dst[i].w)
-                     : "l"(lrow + c));
+      if (c < a.vocab) {
+        if (kEvictFirst)
+          asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(dst[i].x), "=f"(dst[i].y), "=f"(dst[i].z), "=f"(dst[i].w)
+                       : "l"(lrow + c));
+        else
+          asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(dst[i].x), "=f"(dst[i].y), "=f"(dst[i].z), "=f"(dst[i].w)
+                       : "l"(lrow + c));
+      }
     }
   };
   // columns in increasing order: strict comparisons keep the first of equals
@@ -213,13 +204,8 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
   load_batch(x0, 2 * kBatch);
   consume(x1, kBatch);
   load_batch(x1, 3 * kBatch);
-  const int bad = ban_prologue(a, row, col0, ban_bits, hist_s);
-  if (bad) {  // the same in every CTA of the row
-    if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
-    reject_row(a, row, rank);
-    cluster_wait_acquire();  // leave the start-of-kernel phase balanced
-    return;
-  }
+  *bad = ban_prologue(a, row, col0, ban_bits, hist_s);
+  if (*bad) return 0;
   consume(x0, 2 * kBatch);
   consume(x1, 3 * kBatch);
 
@@ -262,10 +248,33 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
       }
     }
   }
-  // (value, column) as one key: larger value first, then the lower column
-  unsigned long long key =
-      bi < a.vocab ? ((unsigned long long)ord_fast(best) << 32) | (0xFFFFFFFFu - (uint32_t)bi)
-                   : 0ull;
+  return bi < a.vocab ? ((unsigned long long)ord_fast(best) << 32) | (0xFFFFFFFFu - (uint32_t)bi)
+                      : 0ull;
+}
+
+// k = 1: the largest masked key of the row, nothing held.
+__global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs in one wave
+    ngram_top1_kernel(const TopkArgs a) {
+  __shared__ uint32_t ban_bits[kChunk / 32];
+  __shared__ unsigned long long warp_best[kWarps];
+  __shared__ unsigned long long cta_best[kMaxTopkCluster];
+  extern __shared__ int32_t hist_s[];
+  const int C = (int)(gridDim.x / (unsigned)a.rows);
+  const int row = (int)(blockIdx.x / (unsigned)C);
+  const int rank = (int)(blockIdx.x % (unsigned)C);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col0 = rank * kChunk;
+  // arrive now, wait before the first remote store: no CTA then writes into a
+  // peer that has not started, and the wait costs nothing by that time
+  cluster_arrive_relaxed();
+  int bad = 0;
+  unsigned long long key = stream_thread_max<true>(a, row, col0, ban_bits, hist_s, &bad);
+  if (bad) {  // the same in every CTA of the row
+    if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
+    reject_row(a, row, rank);
+    cluster_wait_acquire();  // leave the start-of-kernel phase balanced
+    return;
+  }
 #pragma unroll
   for (int off = 16; off; off >>= 1) key = max(key, __shfl_xor_sync(0xffffffffu, key, off));
   if (lane == 0) warp_best[warp] = key;
@@ -289,155 +298,190 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
   }
 }
 
-// k > 1: the row's columns held in registers, radix select over the cluster.
-__global__ void __launch_bounds__(kThreads, 2)
-    ngram_topk_kernel(const TopkArgs a) {
-  __shared__ TopkSmem sm;
-  const int C = (int)(gridDim.x / (unsigned)a.rows);  // cluster size: CTAs per row
-  const int row = (int)(blockIdx.x / (unsigned)C);
-  const int rank = (int)(blockIdx.x % (unsigned)C);
+// Threshold T with exactly k of the n keys (which may repeat) at or above it
+// when the k-th largest key is unique among them, and at least k otherwise:
+// a radix select, 8 bits per pass from the top, stopping when the chosen
+// digit's bin holds exactly the keys still needed.  CTA-wide; keys in shared
+// memory; ends with a barrier.
+__device__ unsigned long long cta_kth_threshold(const unsigned long long *keys, int n, int k,
+                                                uint32_t *hist, uint32_t *scan, uint32_t *sel) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int col0 = rank * kChunk;
-  float *lrow = a.logits + (int64_t)row * a.ld;
-
-  // ---- issue this CTA's loads first (columns col0 + 4 * (tid + 256 i) + u)
-  float4 x[kF4PerThread];
-#pragma unroll
-  for (int i = 0; i < kF4PerThread; ++i) {
-    const int c = col0 + 4 * (tid + kThreads * i);
-    x[i] = c < a.vocab ? __ldcs(reinterpret_cast<const float4 *>(lrow + c))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  sm.hist[0][tid] = 0;
-  if (tid == 0) sm.n_cand = 0;
-  extern __shared__ int32_t hist_s[];
-  stage_history(a, row, hist_s);
-  const int bad = ban_prologue(a, row, col0, sm.ban_bits, hist_s);
-  if (bad) {  // the same in every CTA of the row: all leave before any cluster barrier
-    if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
-    reject_row(a, row, rank);
-    return;
-  }
-
-  // ---- keys: high word = order image of the masked value, low = ~column
-  uint32_t o[kEPT];
-#pragma unroll
-  for (int i = 0; i < kF4PerThread; ++i) {
-    const int c4 = 4 * (tid + kThreads * i);
-    const uint32_t bits = sm.ban_bits[c4 >> 5] >> (c4 & 31);
-    const float v[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool live = col0 + c4 + u < a.vocab;
-      o[4 * i + u] = !live ? 0u : ((bits >> u) & 1u) ? ord_fast(-INFINITY) : ord_fast(v[u]);
-    }
-  }
-  // low word of element e: 2^32 - 1 - column, an immediate offset from nb
-  const uint32_t nb = 0xFFFFFFFFu - (uint32_t)(col0 + 4 * tid);
-  auto key_of = [&](int e) -> unsigned long long {
-    const uint32_t lo = nb - (uint32_t)(4 * kThreads * (e >> 2) + (e & 3));
-    return ((unsigned long long)o[e] << 32) | (unsigned long long)lo;
-  };
-
-  cluster_arrive_relaxed();
-  cluster_wait_acquire();  // every CTA of the cluster has started
-
-  // ---- radix select, 8 bits per pass from the top of the 64-bit key
-  unsigned long long prefix = 0;  // chosen digits so far
-  uint32_t need = (uint32_t)a.k;
+  unsigned long long prefix = 0;
+  uint32_t need = (uint32_t)k;
   int pass = 0;
   for (;; ++pass) {
-    const int buf = pass & 1;
-    const int shift = 56 - 8 * pass;  // this pass's digit
-#pragma unroll
-    for (int e = 0; e < kEPT; ++e) {
-      if (!o[e]) continue;
-      const unsigned long long key = key_of(e);
+    const int shift = 56 - 8 * pass;
+    hist[tid] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+      const unsigned long long key = keys[i];
       if (pass == 0 || (key >> (shift + 8)) == prefix)
-        atomicAdd(&sm.hist[buf][(uint32_t)(key >> shift) & 0xFFu], 1u);
+        atomicAdd(&hist[(uint32_t)(key >> shift) & 0xFFu], 1u);
     }
     __syncthreads();
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    // bin (255 - tid) summed over the cluster; suffix sums = prefix scan of the reversed bins
+    // bin (255 - tid); suffix sums = prefix scan of the reversed bins
     const int bin = 255 - tid;
-    uint32_t cnt = 0;
-    for (int r = 0; r < C; ++r) cnt += ld_cluster_u32(map_to_rank(&sm.hist[buf][bin], r));
-    sm.hist[buf ^ 1][tid] = 0;  // the next pass's buffer (its readers are past this barrier)
+    const uint32_t cnt = hist[bin];
     uint32_t inc = cnt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, inc, off);
       if (lane >= off) inc += y;
     }
-    if (lane == 31) sm.scan[warp] = inc;
+    if (lane == 31) scan[warp] = inc;
     __syncthreads();
     uint32_t before = 0;
-    for (int i = 0; i < warp; ++i) before += sm.scan[i];
+    for (int i = 0; i < warp; ++i) before += scan[i];
     const uint32_t incl = before + inc;  // keys in bins >= bin
     if (incl >= need && incl - cnt < need) {
-      sm.sel_digit = (uint32_t)bin;
-      sm.sel_need = need - (incl - cnt);
-      sm.sel_done = cnt == need - (incl - cnt);
+      sel[0] = (uint32_t)bin;
+      sel[1] = need - (incl - cnt);
+      sel[2] = cnt == need - (incl - cnt);
     }
     __syncthreads();
-    prefix = (prefix << 8) | sm.sel_digit;
-    need = sm.sel_need;
-    if (sm.sel_done || pass == 7) break;
+    prefix = (prefix << 8) | sel[0];
+    need = sel[1];
+    const bool done = sel[2] || pass == 7;
+    __syncthreads();  // sel and hist are rewritten by the next pass
+    if (done) break;
   }
-  // ---- exactly k keys have their top (pass + 1) digits >= prefix
-  const int shift = 56 - 8 * pass;
-  const uint32_t cand_addr = map_to_rank(&sm.cand[0], 0);
-  const uint32_t count_addr = map_to_rank(&sm.n_cand, 0);
+  return prefix << (56 - 8 * pass);
+}
+
+// k > 1, one cluster per row:
+//  1. the streaming pass gives each thread its largest masked key;
+//  2. the leader gathers the C x 256 thread maxima and finds the k-th largest,
+//     T: at least k keys of the row are >= T, and any key >= T lies in one of
+//     the k threads whose maximum is >= T, so at most 64 k keys are;
+//  3. every CTA rereads its columns (from L2) and sends its keys >= T to the
+//     leader;
+//  4. the leader selects the k largest of those candidates exactly, orders
+//     them, writes them and samples.
+__global__ void __launch_bounds__(kThreads, 4)
+    ngram_topk_kernel(const TopkArgs a) {
+  __shared__ uint32_t ban_bits[kChunk / 32];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t scan[kWarps];
+  __shared__ uint32_t sel[3];
+  __shared__ unsigned long long thr;               // T, written by the leader into every CTA
+  __shared__ uint32_t n_cand, n_top;               // leader: candidates received, selected
+  __shared__ unsigned long long sorted[kTopkMax];
+  __shared__ unsigned long long top[kTopkMax];
+  __shared__ float prob[kTopkMax];
+  extern __shared__ __align__(16) uint8_t dyn[];
+  unsigned long long *keybuf = reinterpret_cast<unsigned long long *>(dyn);  // kTopkCandidates
+  int32_t *hist_s = reinterpret_cast<int32_t *>(dyn + kTopkCandidates * 8);
+  const int C = (int)(gridDim.x / (unsigned)a.rows);
+  const int row = (int)(blockIdx.x / (unsigned)C);
+  const int rank = (int)(blockIdx.x % (unsigned)C);
+  const int tid = threadIdx.x;
+  const int col0 = rank * kChunk;
+  const float *lrow = a.logits + (int64_t)row * a.ld;
+  cluster_arrive_relaxed();
+  if (tid == 0) {
+    n_cand = 0;
+    n_top = 0;
+  }
+  int bad = 0;
+  const unsigned long long key = stream_thread_max<false>(a, row, col0, ban_bits, hist_s, &bad);
+  if (bad) {  // the same in every CTA of the row
+    if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
+    reject_row(a, row, rank);
+    cluster_wait_acquire();
+    return;
+  }
+  // ---- 2. thread maxima into the leader; T back to every CTA
+  cluster_wait_acquire();  // every CTA of the cluster has started
+  st_cluster_u64(map_to_rank(&keybuf[rank * kThreads + tid], 0), key);
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  if (rank == 0) {
+    const unsigned long long T = cta_kth_threshold(keybuf, C * kThreads, a.k, hist, scan, sel);
+    if (tid < C) st_cluster_u64(map_to_rank(&thr, tid), T);
+  }
+  cluster_arrive_release();
+  cluster_wait_acquire();
+  // ---- 3. this CTA's keys >= T to the leader (its key buffer is free again)
+  {
+    const unsigned long long T = thr;
+    const uint32_t cand_addr = map_to_rank(keybuf, 0);
+    const uint32_t count_addr = map_to_rank(&n_cand, 0);
+    for (int i0 = 0; i0 < kF4PerThread; i0 += 8) {
+      float4 y[8];
 #pragma unroll
-  for (int e = 0; e < kEPT; ++e) {
-    if (!o[e]) continue;
-    const unsigned long long key = key_of(e);
-    if ((key >> shift) >= prefix) {
-      const uint32_t slot = atom_add_cluster_u32(count_addr, 1u);
-      if (slot < (uint32_t)kTopkMax) st_cluster_u64(cand_addr + 8u * slot, key);
+      for (int i = 0; i < 8; ++i) {
+        const int c = col0 + 4 * (tid + kThreads * (i0 + i));
+        y[i] = c < a.vocab ? *reinterpret_cast<const float4 *>(lrow + c)
+                           : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = col0 + 4 * (tid + kThreads * (i0 + i));
+        const uint32_t bits = ban_bits[(c - col0) >> 5] >> ((c - col0) & 31);
+        const float e[4] = {y[i].x, y[i].y, y[i].z, y[i].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (c + u >= a.vocab) continue;
+          const float vm = ((bits >> u) & 1u) ? -INFINITY : e[u];
+          const unsigned long long kk =
+              ((unsigned long long)ord_fast(vm) << 32) | (0xFFFFFFFFu - (uint32_t)(c + u));
+          if (kk >= T) {
+            const uint32_t slot = atom_add_cluster_u32(count_addr, 1u);
+            if (slot < (uint32_t)kTopkCandidates) st_cluster_u64(cand_addr + 8u * slot, kk);
+          }
+        }
+      }
     }
   }
   cluster_arrive_release();
   cluster_wait_acquire();
-  if (rank != 0) return;
+  if (rank != 0) return;  // the leader reads only its own shared memory from here
 
-  // ---- leader: order the k keys, write them, sample
+  // ---- 4. the k largest candidates, ordered
   const int k = a.k;
-  if (tid < k) {
-    const unsigned long long mine = sm.cand[tid];
-    int r = 0;
-    for (int j = 0; j < k; ++j) r += sm.cand[j] > mine;
-    sm.sorted[r] = mine;
+  const int nc = min((int)n_cand, kTopkCandidates);
+  const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel);
+  for (int i = tid; i < nc; i += kThreads) {
+    const unsigned long long kk = keybuf[i];
+    if (kk >= T2) {
+      const uint32_t slot = atomicAdd(&n_top, 1u);
+      if (slot < (uint32_t)kTopkMax) top[slot] = kk;
+    }
   }
   __syncthreads();
   if (tid < k) {
-    const unsigned long long key = sm.sorted[tid];
-    const int col = (int)(0xFFFFFFFFu - (uint32_t)key);
-    const float val = ord_value((uint32_t)(key >> 32));
+    const unsigned long long mine = top[tid];
+    int r = 0;
+    for (int j = 0; j < k; ++j) r += top[j] > mine;
+    sorted[r] = mine;
+  }
+  __syncthreads();
+  if (tid < k) {
+    const unsigned long long kk = sorted[tid];
+    const int col = (int)(0xFFFFFFFFu - (uint32_t)kk);
+    const float val = ord_value((uint32_t)(kk >> 32));
     a.top_idx[(int64_t)row * k + tid] = col;
     if (a.top_val) a.top_val[(int64_t)row * k + tid] = val;
-    const float x0 = ord_value((uint32_t)(sm.sorted[0] >> 32));
-    sm.prob[tid] = (val == -INFINITY || x0 == -INFINITY) ? 0.f
-                                                        : exp2f((val - x0) * a.inv_temp_log2e);
+    const float x0 = ord_value((uint32_t)(sorted[0] >> 32));
+    prob[tid] = (val == -INFINITY || x0 == -INFINITY) ? 0.f : exp2f((val - x0) * a.inv_temp_log2e);
   }
   __syncthreads();
   if (tid == 0 && a.token) {
     int pick = 0;
-    if (a.uniform && sm.prob[0] > 0.f) {
+    if (a.uniform && prob[0] > 0.f) {
       float total = 0.f;
-      for (int i = 0; i < k; ++i) total += sm.prob[i];
+      for (int i = 0; i < k; ++i) total += prob[i];
       const float target = a.uniform[row] * total;
       float cum = 0.f;
       pick = -1;
       for (int i = 0; i < k; ++i) {
-        if (sm.prob[i] == 0.f) continue;
-        cum += sm.prob[i];
+        if (prob[i] == 0.f) continue;
+        cum += prob[i];
         pick = i;
         if (cum > target) break;
       }
     }
-    a.token[row] = (int)(0xFFFFFFFFu - (uint32_t)sm.sorted[pick]);
+    a.token[row] = (int)(0xFFFFFFFFu - (uint32_t)sorted[pick]);
   }
 }
 
@@ -478,7 +522,15 @@ cudaError_t launch_ngram_topk(float *logits, int64_t ld, const int32_t *history,
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3((unsigned)(rows * C));
   lc.blockDim = dim3(kThreads);
-  lc.dynamicSmemBytes = (size_t)(window > 0 ? window : 1) * sizeof(int32_t);  // the history
+  // the history (and for k > 1 the candidate buffer in front of it)
+  const size_t hist_bytes = (size_t)(window > 0 ? window : 1) * sizeof(int32_t);
+  lc.dynamicSmemBytes = k == 1 ? hist_bytes : (size_t)kTopkCandidates * 8 + hist_bytes;
+  if (k > 1 && lc.dynamicSmemBytes > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(ngram_topk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)lc.dynamicSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
   lc.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
