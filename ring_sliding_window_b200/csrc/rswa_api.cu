@@ -199,6 +199,12 @@ int choose_cluster_size(const rswa_config *c, const int64_t *plen) {
   int64_t max_len = 0;
   for (int b = 0; b < c->batch; ++b) max_len = std::max<int64_t>(max_len, plen[b] + c->window);
   int C = (int)std::min<int64_t>(16, std::max<int64_t>(2, (max_len + 63) / 64));
+  // RSWA_DECODE_CLUSTER=2|4|8|16 sets the cluster size (for measurements)
+  const char *cenv = getenv("RSWA_DECODE_CLUSTER");
+  if (cenv) {
+    const int c = atoi(cenv);
+    if (c == 2 || c == 4 || c == 8 || c == 16) C = c;
+  }
   const int64_t rings = (int64_t)c->batch * c->num_heads;
   for (; C >= 2; C /= 2) {
     const int fit = decode_max_clusters(c->dtype, c->head_dim, C);
