@@ -740,7 +740,7 @@ def run_swa(args, flush, s, hbm_peak):
                 for P in w.prefill_lens)
     res["prefill_standard_swa"] = {"ms_per_layer": statistics.mean(pf_ms),
                                    "tflops": flops / (statistics.mean(pf_ms) / 1e3) / 1e12,
-                                   "kernel": "prefill_simt_kernel (CUDA cores)"}
+                                   "kernel": "prefill_tc_kernel, key tiles of each window only"}
     rig.st.close()
     del rig
     torch.cuda.empty_cache()

@@ -221,17 +221,18 @@ rswa_status rswa_state_set_rope(rswa_state *state, int32_t policy, float theta, 
  * t-th generated token (position P_b + t) to positions P_b + t - W + 1 ..
  * P_b + t, i.e. the last W - 1 - t prompt tokens while t < W - 1 plus the
  * ring.  The cache layout, the ring writes and rswa_advance are unchanged:
- * the mode changes what is attended, not what is stored.  The prefill runs
- * on the CUDA-core kernel; decode gives each ring a cluster of ceil(W / 64)
- * CTAs.
+ * the mode changes what is attended, not what is stored.  The prefill visits
+ * only the key tiles of each query tile's window; decode gives each ring a
+ * cluster of ceil(W / 64) CTAs.
  * ------------------------------------------------------------------------ */
 typedef enum rswa_attention_mode {
   RSWA_ATTN_RING = 0,          /* R-SWA (default) */
   RSWA_ATTN_STANDARD_SWA = 1   /* the window also cuts the prompt */
 } rswa_attention_mode;
 
-/* Host only; takes effect for the calls enqueued after it.  RSWA_EINVAL for
- * an unknown mode. */
+/* Takes effect for the calls enqueued after it.  Switching mode re-uploads
+ * the prefill work list with a synchronous copy (call it before enqueuing
+ * work, not between calls in flight).  RSWA_EINVAL for an unknown mode. */
 rswa_status rswa_state_set_attention(rswa_state *state, int32_t mode);
 
 /* Free the host-side state.  Device memory stays the caller's. */

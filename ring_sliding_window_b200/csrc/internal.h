@@ -146,7 +146,10 @@ cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k,
 
 // Prefill work list of the tensor-core kernel: blocks of two consecutive
 // 128-row query tiles of one (b, h), in launch order.
-std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms);
+// one_tile: one query tile per block (the standard sliding window's blocks
+// have different key ranges per tile).
+std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms,
+                                      bool one_tile = false);
 cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
                          const int32_t *hist_len, int rows, int vocab, int n, int window,
                          int *err, cudaStream_t s);

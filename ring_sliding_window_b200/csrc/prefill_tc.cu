@@ -153,9 +153,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = blk.x, h = blk.y, qt0 = blk.z, ntiles = blk.w;
   const int P = v.plen[b];
   const int tok0 = (int)v.tok_base[b];
-  // key tiles needed by each query tile (causal): 0 .. qt
-  const int n_kv_a = qt0 + 1, n_kv_b = ntiles > 1 ? qt0 + 2 : 0;
-  const int n_kv_all = qt0 + ntiles;
+  // Key tiles j0 .. qt of query tile qt: j0 = 0 (causal), or, for the
+  // standard sliding window, the tile of the first key in the window of the
+  // block's first query (blocks then hold one query tile).  Loops below count
+  // iterations from 0; key tile = j0 + iteration.
+  const int j0 = v.swa ? max(0, qt0 * kTile - v.W + 1) / kTile : 0;
+  const int n_kv_a = qt0 + 1 - j0, n_kv_b = ntiles > 1 ? qt0 + 2 - j0 : 0;
+  const int n_kv_all = qt0 + ntiles - j0;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
@@ -222,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *dst = is_k ? sm.k[s] : sm.v[s];
         if (!wait_bar(empty, ((j / nst) & 1) ^ 1, v.err, dead)) break;
         mbar_arrive_expect_tx(full, kTileBytes);
-        tc::tma_load_2d(dst, tm, x0, y0 + j * kTile, full);
-        tc::tma_load_2d(dst + kHalfBytes, tm, x0 + 64, y0 + j * kTile, full);
+        tc::tma_load_2d(dst, tm, x0, y0 + (j0 + j) * kTile, full);
+        tc::tma_load_2d(dst + kHalfBytes, tm, x0 + 64, y0 + (j0 + j) * kTile, full);
         issued = j + 1;
       }
       // every load issued has landed before the CTA may exit (bounded)
@@ -303,10 +307,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::ld32(t_s + 64, reinterpret_cast<uint32_t *>(s) + 64);
       tc::ld32(t_s + 96, reinterpret_cast<uint32_t *>(s) + 96);
       tc::wait_ld();
-      if (j == qt) {
+      if (j0 + j == qt) {
 #pragma unroll
         for (int c = 0; c < kTile; ++c)
           if (c > r) s[c] = -INFINITY;
+      }
+      if (v.swa) {
+        // keys before the window of query row r: key < query - W + 1
+        const int lim = (qt - j0 - j) * kTile + r - v.W + 1;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (c < lim) s[c] = -INFINITY;
       }
       // row max as an 8-way tree (a single running max would be a 128-deep
       // dependency chain)
@@ -338,7 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) rs4[i] = 0;
       const uint64_t sl2x2 = tc::f2_pack(sl2, sl2);
-      const uint64_t negm2 = tc::f2_pack(-m_use, -m_use);
+      // a row whose keys so far are all outside its window has m = -inf:
+      // its p are 0 (2^-inf), and the next tile's max rescales O and l by 0
+      const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+      const uint64_t negm2 = tc::f2_pack(-m_sub, -m_sub);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];

@@ -123,13 +123,14 @@ DecodePlan plan_decode(const rswa_config *c, const int64_t *plen, const int64_t 
 // one wave of blocks; inside a super-group blocks run longest first.  The
 // CTAs running together then share a few rings' K/V through L2, and the
 // last wave is not left with one long block.
-std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms) {
+std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen, int num_sms,
+                                      bool one_tile) {
   const int B = c->batch, H = c->num_heads;
   // Pairs of tiles halve the K/V traffic per query row, but a batch too
   // small to give every SM a pair runs faster with one tile per CTA.
   int64_t pairs = 0;
   for (int b = 0; b < B; ++b) pairs += (int64_t)H * ((plen[b] + 2 * kPrefillTile - 1) / (2 * kPrefillTile));
-  const int per_block = pairs >= num_sms ? 2 : 1;
+  const int per_block = pairs >= num_sms && !one_tile ? 2 : 1;
   std::vector<int4> out;
   std::vector<int4> group;
   int64_t group_blocks = 0;
@@ -428,9 +429,7 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
   const void *qa = rope ? (const void *)out : q;
   const void *kca = rope ? (const void *)kc : nullptr;
   if (e == cudaSuccess) {
-    // the standard sliding window runs on the CUDA-core kernel (its work,
-    // W keys per query, is too small for the tensor-core pipeline)
-    if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128 && !s->dv.swa)
+    if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128)
       e = launch_prefill_tc(s->dv, qa, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, kca,
                             (int64_t)s->cfg.num_heads * s->pool_slots, st);
     else
@@ -533,7 +532,17 @@ rswa_status rswa_state_set_rope(rswa_state *s, int32_t policy, float theta, void
 rswa_status rswa_state_set_attention(rswa_state *s, int32_t mode) {
   if (!s) return RSWA_EINVAL;
   if (mode != RSWA_ATTN_RING && mode != RSWA_ATTN_STANDARD_SWA) return RSWA_EINVAL;
-  s->dv.swa = mode == RSWA_ATTN_STANDARD_SWA;
+  const bool swa = mode == RSWA_ATTN_STANDARD_SWA;
+  if (swa != (s->dv.swa != 0)) {
+    // re-plan the prefill blocks: one query tile per block with the window
+    if (current_device() != s->device) return RSWA_EINVAL;
+    const std::vector<int4> pf = plan_prefill_blocks(&s->cfg, s->plen.data(), s->num_sms, swa);
+    cudaError_t e = cudaMemcpy((void *)s->dv.pf_blocks, pf.data(), pf.size() * sizeof(int4),
+                               cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return from_cuda(e);
+    s->dv.n_pf_blocks = (int)pf.size();
+  }
+  s->dv.swa = swa;
   // the window holds at most W keys per ring: one cluster of ceil(W / 64)
   // CTAs per ring (clusters are independent, so any batch size runs)
   const char *env = getenv("RSWA_DECODE_SPLIT");
