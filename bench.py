@@ -487,6 +487,8 @@ def run_ours(args, rank, world, local_rank):
                 also.append(run_rope(args, flush, s, hbm_peak, tc_peak))
             elif name == "standard_swa":
                 also.append(run_swa(args, flush, s, hbm_peak))
+            elif name == "keysplit":
+                also.append(run_keysplit(args, flush, s, hbm_peak))
             else:
                 also.append(run_also(synth.workload(name), args, flush, s, hbm_peak, tc_peak))
             torch.cuda.empty_cache()
@@ -749,6 +751,71 @@ def run_swa(args, flush, s, hbm_peak):
     return res
 
 
+def run_keysplit(args, flush, s, hbm_peak, reps=20):
+    """Key-range split of one near-max sequence (prefill_len 32,640, W = 128,
+    10 heads x 128) into G shares, run here one after another on one device:
+    per layer, G partial decode launches plus the merge, against one full
+    decode launch.  On G devices the shares run side by side and only the
+    partials (G x H x (d + 2) floats) cross between them; here the numbers
+    show the split's own cost.  Steady state, L2 flushed before each rep."""
+    from ring_sliding_window_b200 import rswa
+    from ring_sliding_window_b200.keysplit import share_bounds
+    P, W, H, d = 127 * synth.TOKENS_PER_PAGE + 128, 128, 10, 128
+    row = H * d * 2
+    res = {"workload": "keysplit (one sequence, prefill_len 32,640)"}
+    q = torch.randn(1, H, d, device="cuda").to(torch.bfloat16)
+    kn, vn = torch.randn_like(q), torch.randn_like(q)
+
+    def timed(fn):
+        ms = []
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                fn()
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                fn()
+                e1.record(s)
+                ms.append((e0, e1))
+        s.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ms) * 1e3
+
+    for G in (1, 2, 4):
+        bounds = share_bounds(P, G)
+        states = []
+        for g, (lo, hi) in enumerate(bounds):
+            st = rswa.State(1, 1, H, d, W, [hi - lo], dtype=torch.bfloat16, n_generated=[W])
+            gen = torch.Generator(device="cuda").manual_seed(950_100 + g)
+            st.k_cache[0].normal_(generator=gen)
+            st.v_cache[0].normal_(generator=gen)
+            states.append(st)
+        ml = torch.empty(G, 1, H, 2, device="cuda")
+        o = torch.empty(G, 1, H, d, device="cuda")
+        out = torch.empty_like(q)
+
+        def step():
+            for g, st in enumerate(states):
+                lo, hi = bounds[g]
+                st.decode_step_partial(0, q, kn, vn, 0, (hi - lo) + (W if g == G - 1 else 0),
+                                       ml[g], o[g], stream=s)
+            rswa.rswa_combine_partials(ml, o, out, stream=s)
+
+        if G == 1:
+            full = rswa.State(1, 1, H, d, W, [P], dtype=torch.bfloat16, n_generated=[W])
+            full_us = timed(lambda: full.decode_step(0, q, kn, vn, out, stream=s))
+            res["full_decode_us"] = full_us
+            full.close()
+        us = timed(step)
+        nbytes = 2 * (P + W) * row
+        res[f"G{G}"] = {"us_per_layer_all_shares": us, "kv_gbs": nbytes / (us * 1e-6) / 1e9,
+                        "partial_floats_exchanged": G * H * (d + 2)}
+        for st in states:
+            st.close()
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_also(w, args, flush, s, hbm_peak, tc_peak):
     steps = args.also_steps
     rig = DecodeRig(w, w.window, "random", s)
@@ -817,7 +884,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
     ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving,"
-                                      "continuous_batching,ngram_topk,rope,standard_swa")
+                                      "continuous_batching,ngram_topk,rope,standard_swa,"
+                                      "keysplit")
     ap.add_argument("--also-steps", type=int, default=40)
     ap.add_argument("--skip-prefill-also", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -235,6 +235,40 @@ typedef enum rswa_attention_mode {
  * work, not between calls in flight).  RSWA_EINVAL for an unknown mode. */
 rswa_status rswa_state_set_attention(rswa_state *state, int32_t mode);
 
+/* ------------------------------------------------------------------------
+ * Key-range split of one long sequence's cache over G devices.  Softmax
+ * attention over a key set is the log-sum-exp merge of its value over the
+ * parts of any partition of the set, so G shares of the cache can each
+ * produce a partial (m, l, o) and one merge gives the decode output.  A
+ * process per device holds its share as an ordinary state (its slice of the
+ * prompt as prefill_len; the last share also holds the ring), calls
+ * rswa_decode_step_partial, exchanges the partials (G x B x H x (d + 2)
+ * floats, e.g. an all-gather over NCCL), and calls rswa_combine_partials.
+ * The ring write of a step is done by the share whose range holds the slot.
+ * ------------------------------------------------------------------------ */
+
+/* rswa_decode_step restricted to cache slots [key_lo, key_hi) of every ring
+ * (intersected with the entries held), writing the unnormalised partial:
+ *  part_ml : device float [B][H][2]: m (the running max, in log2 units:
+ *            max of scale*log2(e)*q.k) and l = sum 2^(s - m); an empty range
+ *            gives m = -inf, l = 0;
+ *  part_o  : device float [B][H][d]: sum 2^(s - m) v.
+ * The step's ring write happens only if its slot lies in the range.  16-byte
+ * aligned pointers.  RSWA_EINVAL for a bad range or pointer, RSWA_ESTATE as
+ * rswa_decode_step. */
+rswa_status rswa_decode_step_partial(rswa_state *state, int32_t layer, const void *q,
+                                     const void *k_new, const void *v_new, int64_t key_lo,
+                                     int64_t key_hi, float *part_ml, float *part_o,
+                                     void *stream);
+
+/* Merge `shares` partials per ring: part_ml device float [shares][rings][2],
+ * part_o device float [shares][rings][head_dim] -> out [rings][head_dim] of
+ * `dtype` (RSWA_F32 or RSWA_BF16): out = sum_g 2^(m_g - M) o_g /
+ * sum_g 2^(m_g - M) l_g with M = max_g m_g.  rings = B * H. */
+rswa_status rswa_combine_partials(const float *part_ml, const float *part_o, int32_t shares,
+                                  int64_t rings, int32_t head_dim, int32_t dtype, void *out,
+                                  void *stream);
+
 /* Free the host-side state.  Device memory stays the caller's. */
 rswa_status rswa_state_destroy(rswa_state *state);
 

@@ -203,6 +203,30 @@ def ngram_ban(logits: np.ndarray, history: np.ndarray, hist_len, n: int, window:
     return int(rc)
 
 
+def attend_partial(q, k, v, scale: float):
+    """The share of softmax attention over one part of a key set, in FP64:
+    m = max_j s_j with s_j = scale * log2(e) * q.k_j (log2 units),
+    l = sum_j 2^(s_j - m), o = sum_j 2^(s_j - m) v_j.  An empty part gives
+    (-inf, 0, 0).  q: [d]; k, v: [n, d]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    if k.shape[0] == 0:
+        return -np.inf, 0.0, np.zeros(q.shape[-1])
+    s = (k @ q) * float(scale) / np.log(2.0)
+    m = float(np.max(s))
+    p = np.exp2(s - m)
+    return m, float(p.sum()), p @ v
+
+
+def combine_partials(parts):
+    """Log-sum-exp merge of (m, l, o) shares: sum 2^(m_g - M) o_g over
+    sum 2^(m_g - M) l_g, M = max m_g; equals attention over the union of the
+    parts (the key-range split of the decode step)."""
+    M = max(m for m, _, _ in parts)
+    w = [0.0 if m == -np.inf else 2.0 ** (m - M) for m, _, _ in parts]
+    L = sum(wi * l for wi, (_, l, _) in zip(w, parts))
+    return sum(wi * o for wi, (_, _, o) in zip(w, parts)) / L
+
+
 def prefill_window(q, k, v, scale: float, window: int) -> np.ndarray:
     """Standard sliding-window prefill, the contrast of "开源5天Star破万之后：
     百度Unlimited-OCR的爆火路径复盘" §2.1 (a standard window would cut the

@@ -108,33 +108,41 @@ __device__ __forceinline__ void rope_lane(float *x, int li, const float2 *cs) {
 }
 
 // This step's key range of a piece, read after the grid-dependency wait:
-// [kb, ke) clipped to the cache entries held (P_b + min(t_b + 1, W)) and,
-// for the standard sliding window, to the slots of the last W positions,
-// [max(0, min(P_b, P_b + t_b - W + 1)), held).  A cluster CTA (rank of C)
-// re-splits that window evenly.  wslot: this step's ring slot, or -1 when
-// the piece lies wholly in the prompt (ring mode only).
+// [kb, ke) clipped to the cache entries held (P_b + min(t_b + 1, W)), for the
+// standard sliding window to the slots of the last W positions,
+// [max(0, min(P_b, P_b + t_b - W + 1)), held), and to the caller's slot range
+// [key_lo, key_hi) of a partial step.  A cluster CTA (rank of C) re-splits
+// that window evenly.  wslot: this step's ring slot, or -1 when the piece
+// lies wholly in the prompt (full ring mode only).
 struct KeyRange {
   int kb, ke, wslot;
 };
 __device__ __forceinline__ KeyRange resolve_range(const DeviceView &v, const DecodePiece &pc,
                                                   int rank, int C) {
   KeyRange r{pc.key_begin, pc.key_end, -1};
-  if (!v.swa && r.ke <= pc.plen) return r;  // no ring counter needed
+  const bool windowed = v.swa || v.key_lo > 0 || v.key_hi < pc.plen + v.W;
+  if (!windowed && r.ke <= pc.plen) return r;  // no ring counter needed
   const int64_t t = v.t[pc.b];
-  const int valid = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);
+  int hi = pc.plen + (int)(t + 1 < (int64_t)v.W ? t + 1 : (int64_t)v.W);  // entries held
   r.wslot = pc.plen + (int)(t % v.W);
-  if (v.swa) {
-    const int64_t lo64 = (int64_t)pc.plen + t - v.W + 1;
-    const int lo = lo64 < 0 ? 0 : (lo64 > pc.plen ? pc.plen : (int)lo64);
+  if (windowed) {
+    int lo = 0;
+    if (v.swa) {
+      const int64_t lo64 = (int64_t)pc.plen + t - v.W + 1;
+      lo = lo64 < 0 ? 0 : (lo64 > pc.plen ? pc.plen : (int)lo64);
+    }
+    lo = max(lo, v.key_lo);  // the caller's key range (a share of a split cache)
+    hi = min(hi, v.key_hi);
+    if (lo > hi) lo = hi;
     if (C > 0) {
-      const int per = (valid - lo + C - 1) / C;
-      r.kb = min(lo + rank * per, valid);
-      r.ke = min(lo + (rank + 1) * per, valid);
+      const int per = (hi - lo + C - 1) / C;
+      r.kb = min(lo + rank * per, hi);
+      r.ke = min(lo + (rank + 1) * per, hi);
     } else {
       r.kb = max(r.kb, lo);
     }
   }
-  r.ke = min(r.ke, valid);
+  r.ke = min(r.ke, hi);
   return r;
 }
 
@@ -145,6 +153,19 @@ struct DecodeArgs {
   void *out;
 };
 
+
+// Element tid of ring bh's result: the normalised output, or, for a partial
+// step, the unnormalised (m, l, o) the caller combines with other shares.
+template <typename T, int D>
+__device__ __forceinline__ void store_result(const DeviceView &v, const DecodeArgs &a, int bh,
+                                             int tid, float m, float l, float acc) {
+  if (v.out_ml) {
+    v.out_o[(int64_t)bh * D + tid] = acc;
+    if (tid == 0) v.out_ml[bh] = make_float2(m, l);
+  } else {
+    ((T *)a.out)[(int64_t)bh * D + tid] = from_float<T>(acc / l);
+  }
+}
 
 // kCluster = false: stream-K pieces from the work tables, partials merged
 //   through global memory by the CTA that finishes a ring last.
@@ -215,8 +236,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   // RSWA_DEVERR_TIMEOUT and the kernel still finishes.  The flag is written by
   // a host copy, which a kernel launched after it never overlaps.
   const bool drop_copies = (*v.fault & RSWA_FAULT_DROP_DECODE_COPIES) != 0;
-  // (The standard-sliding-window mode picks its keys from t_b: no prefetch.)
-  if (warp == S::kConsumerWarps && lane == 0 && !drop_copies && !v.swa) {
+  // (The standard-sliding-window mode picks its keys from t_b and a partial
+  // step clips them to a slot range: no prefetch in either.)
+  const bool prefetch_ok = !v.swa && v.key_lo == 0 && v.out_ml == nullptr;
+  if (warp == S::kConsumerWarps && lane == 0 && !drop_copies && prefetch_ok) {
     const DecodePiece &pc = first_piece;
     const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
     const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
@@ -454,12 +477,13 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         float Mg = -INFINITY;
         for (int r = 0; r < C; ++r) Mg = fmaxf(Mg, sm.cl_ml[r].x);
         float Lg = 0.f, acc = 0.f;
-        for (int r = 0; r < C; ++r) {
-          const float wgt = exp2f(sm.cl_ml[r].x - Mg);  // 0 for an empty range
-          Lg = fmaf(wgt, sm.cl_ml[r].y, Lg);
-          acc = fmaf(wgt, sm.cl_o[r][tid], acc);
-        }
-        ((T *)a.out)[((int64_t)pc.b * v.H + pc.h) * D + tid] = from_float<T>(acc / Lg);
+        if (Mg != -INFINITY)
+          for (int r = 0; r < C; ++r) {
+            const float wgt = exp2f(sm.cl_ml[r].x - Mg);  // 0 for an empty range
+            Lg = fmaf(wgt, sm.cl_ml[r].y, Lg);
+            acc = fmaf(wgt, sm.cl_o[r][tid], acc);
+          }
+        store_result<T, D>(v, a, pc.b * v.H + pc.h, tid, Mg, Lg, acc);
       }
       continue;  // a cluster CTA has exactly one piece
     }
@@ -516,7 +540,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         }
         Mg = Mc;
       }
-      if (tid < D) ((T *)a.out)[(int64_t)bh * D + tid] = from_float<T>(acc / Lg);
+      if (tid < D) store_result<T, D>(v, a, bh, tid, Mg, Lg, acc);
     }
   }
 }
@@ -629,6 +653,36 @@ cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
   }
   if (v.D == 128) return launch_decode_d<float, 128>(v, q, k_new, v_new, kc, vc, out, s, pdl);
   return launch_decode_d<float, 64>(v, q, k_new, v_new, kc, vc, out, s, pdl);
+}
+
+// Log-sum-exp merge of `shares` partials (m, l, o) per ring: one CTA per ring,
+// one thread per output element.
+template <typename T>
+__global__ void combine_kernel(const float2 *__restrict__ ml, const float *__restrict__ o,
+                               int shares, int64_t rings, int D, T *__restrict__ out) {
+  const int64_t bh = blockIdx.x;
+  const int e = threadIdx.x;
+  float Mg = -INFINITY;
+  for (int g = 0; g < shares; ++g) Mg = fmaxf(Mg, ml[(int64_t)g * rings + bh].x);
+  float Lg = 0.f, acc = 0.f;
+  if (Mg != -INFINITY)
+    for (int g = 0; g < shares; ++g) {
+      const float2 p = ml[(int64_t)g * rings + bh];
+      const float wgt = exp2f(p.x - Mg);  // 0 for an empty share
+      Lg = fmaf(wgt, p.y, Lg);
+      acc = fmaf(wgt, o[((int64_t)g * rings + bh) * D + e], acc);
+    }
+  out[bh * D + e] = from_float<T>(acc / Lg);
+}
+
+cudaError_t launch_combine(const float2 *ml, const float *o, int shares, int64_t rings, int D,
+                           int dtype, void *out, cudaStream_t s) {
+  if (dtype == RSWA_BF16)
+    combine_kernel<__nv_bfloat16><<<(unsigned)rings, D, 0, s>>>(ml, o, shares, rings, D,
+                                                                (__nv_bfloat16 *)out);
+  else
+    combine_kernel<float><<<(unsigned)rings, D, 0, s>>>(ml, o, shares, rings, D, (float *)out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s) {

@@ -13,6 +13,7 @@
 // rswa_decode_step, with the scratch taken from a file-scope __device__ array
 // of a fixed size (kNoAllocScratchBytes per device, held until the process
 // exits).  The caller still passes the cache, inputs and outputs.
+#include <climits>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <string.h>
@@ -106,6 +107,7 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
 
   DeviceView v;
   memset(&v, 0, sizeof(v));
+  v.key_hi = INT_MAX;  // the whole cache
   v.B = B;
   v.H = cfg->num_heads;
   v.D = cfg->head_dim;

@@ -87,6 +87,9 @@ struct DeviceView {
   int n_pieces;
   int cluster_size;  // > 0: decode runs one ring per cluster of this many CTAs
   int swa;           // 1: standard sliding window (the window also cuts the prompt)
+  int key_lo, key_hi;  // slot range a decode step attends to (a share of a split cache)
+  float2 *out_ml;      // non-null: write (m, l) [B*H] and o [B*H][D] instead of out
+  float *out_o;
   int rope;          // rswa_rope_policy (0: keys and queries used as given)
   float rope_theta;
   float2 *rope_cs;   // [B][D/2] (cos, sin) of the position of each request's next token
@@ -123,6 +126,8 @@ cudaError_t launch_decode(const DeviceView &v, const void *q, const void *k_new,
                           const void *v_new, void *kc, void *vc, void *out, cudaStream_t s,
                           bool pdl);
 cudaError_t launch_advance(const DeviceView &v, cudaStream_t s);
+cudaError_t launch_combine(const float2 *ml, const float *o, int shares, int64_t rings, int D,
+                           int dtype, void *out, cudaStream_t s);
 cudaError_t launch_ngram_topk(float *logits, int64_t ld, const int32_t *history, int64_t hist_ld,
                               const int32_t *hist_len, int rows, int vocab, int n, int window,
                               int k, int mask_in_place, const float *uniform, float temperature,

@@ -1,5 +1,6 @@
 // librswa host layer: argument checks, the split-K work plan, the workspace
 // layout, and the exported C entry points declared in include/rswa.h.
+#include <climits>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdlib.h>
@@ -189,16 +190,20 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 // Decode split for this batch: 0 = stream-K pieces merged through global
 // memory; C > 0 = one ring per cluster of C CTAs merged through distributed
 // shared memory.  The cluster form is used when every ring's cluster can be
-// resident at once (small batches, where the global hand-off dominates).
+// resident at once and gives at least half the CTAs stream-K would (small
+// batches of short rings, where the global hand-off dominates).
 // RSWA_DECODE_SPLIT=streamk|cluster overrides the choice (the cluster form
 // still needs the clusters to fit).
-int choose_cluster_size(const rswa_config *c, const int64_t *plen) {
+int choose_cluster_size(const rswa_config *c, const int64_t *plen, int num_sms) {
   const char *env = getenv("RSWA_DECODE_SPLIT");
   const bool force_streamk = env && strcmp(env, "streamk") == 0;
   const bool force_cluster = env && strcmp(env, "cluster") == 0;
   if (force_streamk) return 0;
-  int64_t max_len = 0;
-  for (int b = 0; b < c->batch; ++b) max_len = std::max<int64_t>(max_len, plen[b] + c->window);
+  int64_t max_len = 0, rows = 0;
+  for (int b = 0; b < c->batch; ++b) {
+    max_len = std::max<int64_t>(max_len, plen[b] + c->window);
+    rows += (plen[b] + c->window) * c->num_heads;
+  }
   int C = (int)std::min<int64_t>(16, std::max<int64_t>(2, (max_len + 63) / 64));
   // RSWA_DECODE_CLUSTER=2|4|8|16 sets the cluster size (for measurements)
   const char *cenv = getenv("RSWA_DECODE_CLUSTER");
@@ -207,6 +212,12 @@ int choose_cluster_size(const rswa_config *c, const int64_t *plen) {
     if (c == 2 || c == 4 || c == 8 || c == 16) C = c;
   }
   const int64_t rings = (int64_t)c->batch * c->num_heads;
+  // a few long rings need more CTAs than 16 per ring: stream-K spreads them
+  // over the whole GPU (the merge then costs little next to the stream)
+  const int64_t streamk_grid =
+      std::min<int64_t>((int64_t)num_sms * decode_ctas_per_sm(c->dtype, c->head_dim),
+                        (rows + kMinRowsPerCta - 1) / kMinRowsPerCta);
+  if (!force_cluster && rings * C * 2 < streamk_grid) return 0;
   for (; C >= 2; C /= 2) {
     const int fit = decode_max_clusters(c->dtype, c->head_dim, C);
     if (fit >= rings) break;
@@ -383,8 +394,12 @@ rswa_status rswa_state_create_pooled(const rswa_config *cfg, const int64_t *pref
   v.part_o = (float *)(w + s->ws.part_o);
   v.decode_grid = s->plan.grid;
   v.n_pieces = s->plan.n_pieces;
-  v.cluster_size = choose_cluster_size(cfg, prefill_len);
+  v.cluster_size = choose_cluster_size(cfg, prefill_len, s->num_sms);
   v.swa = 0;
+  v.key_lo = 0;
+  v.key_hi = INT_MAX;  // the whole cache
+  v.out_ml = nullptr;
+  v.out_o = nullptr;
   v.rope = RSWA_ROPE_NONE;
   v.rope_theta = 10000.f;
   v.rope_cs = (float2 *)(w + s->ws.rope_cs);
@@ -450,6 +465,38 @@ rswa_status rswa_decode_step(rswa_state *s, int32_t layer, const void *q, const 
   if (current_device() != s->device) return RSWA_EINVAL;
   return from_cuda(launch_decode(s->dv, q, k_new, v_new, s->k_cache[(size_t)layer],
                                  s->v_cache[(size_t)layer], out, (cudaStream_t)stream, true));
+}
+
+rswa_status rswa_decode_step_partial(rswa_state *s, int32_t layer, const void *q,
+                                     const void *k_new, const void *v_new, int64_t key_lo,
+                                     int64_t key_hi, float *part_ml, float *part_o,
+                                     void *stream) {
+  if (!s || layer < 0 || layer >= s->cfg.num_layers) return RSWA_EINVAL;
+  if (!q || !k_new || !v_new || !part_ml || !part_o) return RSWA_EINVAL;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(part_ml) ||
+      !aligned16(part_o))
+    return RSWA_EINVAL;
+  if (key_lo < 0 || key_hi < key_lo) return RSWA_EINVAL;
+  if (!s->layer_ready[(size_t)layer]) return RSWA_ESTATE;
+  if (current_device() != s->device) return RSWA_EINVAL;
+  DeviceView v = s->dv;
+  v.key_lo = (int)std::min<int64_t>(key_lo, INT_MAX);
+  v.key_hi = (int)std::min<int64_t>(key_hi, INT_MAX);
+  v.out_ml = reinterpret_cast<float2 *>(part_ml);
+  v.out_o = part_o;
+  return from_cuda(launch_decode(v, q, k_new, v_new, s->k_cache[(size_t)layer],
+                                 s->v_cache[(size_t)layer], nullptr, (cudaStream_t)stream, true));
+}
+
+rswa_status rswa_combine_partials(const float *part_ml, const float *part_o, int32_t shares,
+                                  int64_t rings, int32_t head_dim, int32_t dtype, void *out,
+                                  void *stream) {
+  if (shares < 1 || rings < 0 || (head_dim != 64 && head_dim != 128)) return RSWA_EINVAL;
+  if (dtype != RSWA_F32 && dtype != RSWA_BF16) return RSWA_EINVAL;
+  if (rings == 0) return RSWA_OK;
+  if (!part_ml || !part_o || !out) return RSWA_EINVAL;
+  return from_cuda(launch_combine(reinterpret_cast<const float2 *>(part_ml), part_o, shares, rings,
+                                  head_dim, dtype, out, (cudaStream_t)stream));
 }
 
 rswa_status rswa_advance(rswa_state *s, void *stream) {
@@ -550,7 +597,7 @@ rswa_status rswa_state_set_attention(rswa_state *s, int32_t mode) {
   if (s->dv.swa && !force_streamk)
     s->dv.cluster_size = std::max(1, std::min(16, (s->cfg.window + 63) / 64));
   else
-    s->dv.cluster_size = choose_cluster_size(&s->cfg, s->plen.data());
+    s->dv.cluster_size = choose_cluster_size(&s->cfg, s->plen.data(), s->num_sms);
   return RSWA_OK;
 }
 

@@ -34,7 +34,7 @@ EXPORTED = (
     "rswa_decode_launch_shape", "rswa_pool_create", "rswa_pool_destroy", "rswa_pool_alloc",
     "rswa_pool_free", "rswa_pool_stats", "rswa_pool_capacity", "rswa_pool_cache_bytes",
     "rswa_state_create_pooled", "rswa_ngram_topk", "rswa_state_set_rope",
-    "rswa_state_set_attention",
+    "rswa_state_set_attention", "rswa_decode_step_partial", "rswa_combine_partials",
 )
 RSWA_ATTN_RING, RSWA_ATTN_STANDARD_SWA = 0, 1
 RSWA_ROPE_NONE, RSWA_ROPE_ABSOLUTE, RSWA_ROPE_SLOT = 0, 1, 2
@@ -89,6 +89,10 @@ lib.rswa_check_device_error.argtypes = [_vp, _vp]
 lib.rswa_decode_launch_shape.argtypes = [_vp, _i32p, _i32p]
 lib.rswa_state_set_rope.argtypes = [_vp, ctypes.c_int32, ctypes.c_float, _vp]
 lib.rswa_state_set_attention.argtypes = [_vp, ctypes.c_int32]
+lib.rswa_decode_step_partial.argtypes = [_vp, ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int64,
+                                         ctypes.c_int64, _vp, _vp, _vp]
+lib.rswa_combine_partials.argtypes = [_vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                      ctypes.c_int32, _vp, _vp]
 lib.rswa_ngram_topk.argtypes = [_vp, ctypes.c_int64, _vp, ctypes.c_int64, _vp, ctypes.c_int32,
                                 ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                 ctypes.c_int32, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _vp]
@@ -117,7 +121,7 @@ for _n in ("rswa_state_create", "rswa_state_destroy", "rswa_prefill", "rswa_deco
            "rswa_check_device_error", "rswa_decode_launch_shape", "rswa_pool_create",
            "rswa_pool_destroy", "rswa_pool_alloc", "rswa_pool_free", "rswa_pool_stats",
            "rswa_state_create_pooled", "rswa_ngram_topk", "rswa_state_set_rope",
-           "rswa_state_set_attention"):
+           "rswa_state_set_attention", "rswa_decode_step_partial", "rswa_combine_partials"):
     getattr(lib, _n).restype = ctypes.c_int
 
 
@@ -308,6 +312,25 @@ def rswa_state_set_attention(state, mode: int) -> None:
     _check(lib.rswa_state_set_attention(state, int(mode)), "rswa_state_set_attention")
 
 
+def rswa_decode_step_partial(state, layer, q, k_new, v_new, key_lo, key_hi, part_ml, part_o,
+                             stream=None) -> None:
+    """Decode over cache slots [key_lo, key_hi): part_ml float32 [B, H, 2] (m, l),
+    part_o float32 [B, H, d] (unnormalised)."""
+    _check(lib.rswa_decode_step_partial(state, layer, _ptr(q), _ptr(k_new), _ptr(v_new),
+                                        int(key_lo), int(key_hi), _ptr(part_ml), _ptr(part_o),
+                                        _stream(stream)), "rswa_decode_step_partial")
+
+
+def rswa_combine_partials(part_ml, part_o, out, stream=None) -> None:
+    """part_ml [G, B, H, 2], part_o [G, B, H, d] (float32) -> out [B, H, d]."""
+    G = part_ml.shape[0]
+    rings = part_ml[0].numel() // 2
+    d = part_o.shape[-1]
+    dt = RSWA_BF16 if out.dtype == torch.bfloat16 else RSWA_F32
+    _check(lib.rswa_combine_partials(_ptr(part_ml), _ptr(part_o), G, rings, d, dt, _ptr(out),
+                                     _stream(stream)), "rswa_combine_partials")
+
+
 def rswa_decode_launch_shape(state):
     """(grid, cluster_size) of this state's decode launches; cluster_size 0 = stream-K split."""
     g, c = ctypes.c_int32(0), ctypes.c_int32(0)
@@ -413,6 +436,11 @@ class State:
 
     def set_attention(self, mode: int):
         rswa_state_set_attention(self.handle, mode)
+
+    def decode_step_partial(self, layer, q, k_new, v_new, key_lo, key_hi, part_ml, part_o,
+                            stream=None):
+        rswa_decode_step_partial(self.handle, layer, q, k_new, v_new, key_lo, key_hi, part_ml,
+                                 part_o, stream)
 
 
 class TokenPool:
