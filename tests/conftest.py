@@ -6,6 +6,9 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+# the oracle-mutant tests run the pins against a planted copy of the oracle
+if os.environ.get("RSWA_ORACLE_DIR"):
+    sys.path.insert(0, os.environ["RSWA_ORACLE_DIR"])
 
 
 def pytest_configure(config):
