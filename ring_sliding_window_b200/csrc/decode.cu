@@ -58,11 +58,22 @@ struct DecodeShape {
   static_assert(kEPL * 8 == D, "lane split must cover the row");
 };
 
+// Stages of the shared-memory ring.  The cluster form serves short key
+// ranges (a ring split 16 ways): three stages hold a CTA's whole range, and
+// the smaller footprint lets three CTAs share an SM, so the next layer's
+// CTAs become resident -- and request their prompt rows -- while this
+// layer's are still running.
+template <typename T, int D, bool kCluster>
+constexpr int decode_stages() {
+  return kCluster ? 3 : DecodeShape<T, D>::kStages;
+}
+
 template <typename T, int D, bool kCluster>
 struct __align__(128) DecodeSmem {
   using S = DecodeShape<T, D>;
-  uint8_t k[S::kStages][S::kStageRows * S::kRowBytes];
-  uint8_t v[S::kStages][S::kStageRows * S::kRowBytes];
+  static constexpr int NST = decode_stages<T, D, kCluster>();
+  uint8_t k[NST][S::kStageRows * S::kRowBytes];
+  uint8_t v[NST][S::kStageRows * S::kRowBytes];
   uint8_t sub_k[S::kRowBytes];
   uint8_t sub_v[S::kRowBytes];
   float red_o[S::kGroups][D];
@@ -73,8 +84,8 @@ struct __align__(128) DecodeSmem {
   // leader's copy through distributed shared memory
   float cl_o[kCluster ? kMaxCluster : 1][D];
   float2 cl_ml[kCluster ? kMaxCluster : 1];
-  uint64_t full[S::kStages];
-  uint64_t empty[S::kStages];
+  uint64_t full[NST];
+  uint64_t empty[NST];
 };
 
 // Rotate this lane's slice of a row (rotate-half RoPE, pairs (i, i + D/2))
@@ -179,6 +190,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   using S = DecodeShape<T, D>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem<T, D, kCluster> &sm = *reinterpret_cast<DecodeSmem<T, D, kCluster> *>(smem_raw);
+  constexpr int NST = decode_stages<T, D, kCluster>();
   const DeviceView &v = a.v;
 
   const int warp = threadIdx.x >> 5;
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   }
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S::kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], S::kConsumerWarps);
     }
@@ -243,7 +255,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
     const DecodePiece &pc = first_piece;
     const uint8_t *kbase = (const uint8_t *)a.kc + pc.row0 * S::kRowBytes;
     const uint8_t *vbase = (const uint8_t *)a.vc + pc.row0 * S::kRowBytes;
-    for (int k0 = pc.key_begin; k0 < pc.key_end && pre_stages < S::kStages;
+    for (int k0 = pc.key_begin; k0 < pc.key_end && pre_stages < NST;
          k0 += S::kStageRows) {
       const int rows = (pc.key_end - k0) < S::kStageRows ? (pc.key_end - k0) : S::kStageRows;
       if (k0 + rows > pc.plen) break;
@@ -263,8 +275,8 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
   if (warp == S::kConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane != 0 || drop_copies) return;
-    int stage = pre_stages % S::kStages;
-    uint32_t round = pre_stages / S::kStages;
+    int stage = pre_stages % NST;
+    uint32_t round = pre_stages / NST;
     bool dead = false;
     for (int p = p_begin; p < p_end && !dead; ++p) {
       const DecodePiece pc = p == p_begin ? first_piece : v.pieces[p];
@@ -283,7 +295,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
         mbar_arrive_expect_tx(&sm.full[stage], 2 * bytes);
         bulk_g2s(sm.k[stage], kbase + (int64_t)k0 * S::kRowBytes, bytes, &sm.full[stage]);
         bulk_g2s(sm.v[stage], vbase + (int64_t)k0 * S::kRowBytes, bytes, &sm.full[stage]);
-        if (++stage == S::kStages) {
+        if (++stage == NST) {
           stage = 0;
           ++round;
         }
@@ -436,7 +448,7 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[stage]);
-      if (++stage == S::kStages) {
+      if (++stage == NST) {
         stage = 0;
         ++round;
       }

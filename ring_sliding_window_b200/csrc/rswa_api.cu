@@ -205,11 +205,11 @@ int choose_cluster_size(const rswa_config *c, const int64_t *plen, int num_sms) 
     rows += (plen[b] + c->window) * c->num_heads;
   }
   int C = (int)std::min<int64_t>(16, std::max<int64_t>(2, (max_len + 63) / 64));
-  // RSWA_DECODE_CLUSTER=2|4|8|16 sets the cluster size (for measurements)
+  // RSWA_DECODE_CLUSTER=2..16 sets the cluster size (for measurements)
   const char *cenv = getenv("RSWA_DECODE_CLUSTER");
   if (cenv) {
     const int c = atoi(cenv);
-    if (c == 2 || c == 4 || c == 8 || c == 16) C = c;
+    if (c >= 2 && c <= 16) C = c;
   }
   const int64_t rings = (int64_t)c->batch * c->num_heads;
   // a few long rings need more CTAs than 16 per ring: stream-K spreads them
