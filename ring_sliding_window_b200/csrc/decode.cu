@@ -399,7 +399,9 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
 #pragma unroll
         for (int ps = 0; ps < S::kPasses; ++ps) {
           const int r = ps * S::kGroups + g;
-          float acc = 0.f;
+          // four independent partial sums: a 16-deep FMA chain would be the
+          // latency of every row
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
           if (r < rows) {
             const uint8_t *krow = (owner && k0 + r == wslot) ? sm.sub_k : ks + r * S::kRowBytes;
 #pragma unroll
@@ -409,9 +411,10 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
               Chunk<T>::widen(u, kf);
 #pragma unroll
               for (int e = 0; e < S::kElemPerChunk; ++e)
-                acc = fmaf(qf[j * S::kElemPerChunk + e], kf[e], acc);
+                a4[e & 3] = fmaf(qf[j * S::kElemPerChunk + e], kf[e], a4[e & 3]);
             }
           }
+          float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
           acc += __shfl_xor_sync(0xffffffffu, acc, 1);
           acc += __shfl_xor_sync(0xffffffffu, acc, 2);
           acc += __shfl_xor_sync(0xffffffffu, acc, 4);
