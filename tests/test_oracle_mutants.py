@@ -31,18 +31,38 @@ MUTANTS = [
 ]
 
 
-@pytest.mark.slow
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pins_catch_mutant(tmp_path, name, old, new):
+def _run_mutant(tmp, name, old, new):
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation anchor for {name} not found once"
-    mut = tmp_path / "oracle_mut.c"
-    mut.write_text(src.replace(old, new))
-    so = tmp_path / "liboracle_mut.so"
-    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", str(mut), "-o", str(so),
-                    "-lm"], check=True)
-    env = dict(os.environ, ORACLE_LIB_OVERRIDE=str(so), OMP_NUM_THREADS="2")
+    if src.count(old) != 1:
+        return None, f"mutation anchor for {name} not found once"
+    d = os.path.join(tmp, name)
+    os.makedirs(d)
+    mut = os.path.join(d, "oracle_mut.c")
+    with open(mut, "w") as f:
+        f.write(src.replace(old, new))
+    so = os.path.join(d, "liboracle_mut.so")
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fopenmp", mut, "-o", so, "-lm"],
+                   check=True)
+    env = dict(os.environ, ORACLE_LIB_OVERRIDE=so, OMP_NUM_THREADS="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    """Every mutant's pin run, the runs side by side (one process each)."""
+    import concurrent.futures as cf
+    tmp = str(tmp_path_factory.mktemp("mutants"))
+    with cf.ThreadPoolExecutor(max_workers=min(len(MUTANTS), os.cpu_count() or 1)) as ex:
+        futs = {m[0]: ex.submit(_run_mutant, tmp, *m) for m in MUTANTS}
+        return {k: f.result() for k, f in futs.items()}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_pins_catch_mutant(mutant_runs, name):
+    rc, out = mutant_runs[name]
+    assert rc is not None, out
+    assert rc != 0, f"pins did not catch mutant {name}:\n{out}"

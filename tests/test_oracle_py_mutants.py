@@ -44,16 +44,31 @@ def _run_pins(tmp_path, pins, old=None, new=None):
         src = src.replace(old, new)
     # a marker the pins' process can see: proves the copy is the one imported
     init.write_text(src + "\nPLANTED_COPY = True\n")
-    env = dict(os.environ, RSWA_ORACLE_DIR=str(tmp_path), OMP_NUM_THREADS="2")
+    env = dict(os.environ, RSWA_ORACLE_DIR=str(tmp_path), OMP_NUM_THREADS="1")
     return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                            "-k", "not gloo", os.path.join(ROOT, "tests", pins)],
                           env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
 
 
+@pytest.fixture(scope="module")
+def runs(tmp_path_factory):
+    """The control run and every mutant's pin run, side by side."""
+    import concurrent.futures as cf
+    jobs = [("control", None, None, "test_oracle_rope_pins.py")] + list(MUTANTS)
+    with cf.ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        futs = {name: ex.submit(_run_pins, tmp_path_factory.mktemp(name), pins, old, new)
+                for name, old, new, pins in jobs}
+        return {k: f.result() for k, f in futs.items()}
+
+
 @pytest.mark.slow
-def test_unplanted_copy_passes_and_is_the_one_imported(tmp_path):
-    r = _run_pins(tmp_path, "test_oracle_rope_pins.py")
+def test_unplanted_copy_passes_and_is_the_one_imported(runs, tmp_path):
+    r = runs["control"]
     assert r.returncode == 0, r.stdout[-2000:]
+    dst = tmp_path / "oracle"
+    shutil.copytree(PKG, dst, ignore=shutil.ignore_patterns("__pycache__"))
+    init = dst / "__init__.py"
+    init.write_text(init.read_text() + "\nPLANTED_COPY = True\n")
     env = dict(os.environ, RSWA_ORACLE_DIR=str(tmp_path))
     probe = subprocess.run([sys.executable, "-c",
                             "import sys, os; sys.path.insert(0, os.environ['RSWA_ORACLE_DIR']); "
@@ -63,8 +78,8 @@ def test_unplanted_copy_passes_and_is_the_one_imported(tmp_path):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,old,new,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pins_catch_python_mutant(tmp_path, name, old, new, pins):
-    r = _run_pins(tmp_path, pins, old, new)
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_pins_catch_python_mutant(runs, name):
+    r = runs[name]
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout, r.stdout[-2000:]  # a failing pin, not a broken import
