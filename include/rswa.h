@@ -245,6 +245,9 @@ rswa_status rswa_state_set_attention(rswa_state *state, int32_t mode);
  * rswa_decode_step_partial, exchanges the partials (G x B x H x (d + 2)
  * floats, e.g. an all-gather over NCCL), and calls rswa_combine_partials.
  * The ring write of a step is done by the share whose range holds the slot.
+ * RoPE in the library follows each state's own positions, so a split
+ * sequence rotates its keys and queries before the calls (or all shares but
+ * the first would rotate at shifted positions).
  * ------------------------------------------------------------------------ */
 
 /* rswa_decode_step restricted to cache slots [key_lo, key_hi) of every ring

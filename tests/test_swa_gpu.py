@@ -82,3 +82,43 @@ def test_attention_mode_switch_and_errors():
     assert st.decode_launch_shape()[1] == 1  # ceil(8 / 64) CTAs per ring
     st.set_attention(rswa.RSWA_ATTN_RING)
     assert st.decode_launch_shape() == ring_shape
+
+
+@pytest.mark.parametrize("policy", [1, 2])
+def test_standard_swa_with_rope(policy):
+    """The two options compose: rotated keys in the cache, a window over them."""
+    from ring_sliding_window_b200 import rswa
+    dtype, d, B, H, W, P, steps, theta = torch.bfloat16, 128, 2, 2, 8, (200, 37), 14, 10000.0
+    w = synth.Workload("swa_rope", 91 + policy, dtype, B, 1, H, d, W, P, steps)
+    st = rswa.State(B, 1, H, d, W, P, dtype=dtype)
+    st.set_attention(rswa.RSWA_ATTN_STANDARD_SWA)
+    st.set_rope(policy, theta)
+    pol = "absolute" if policy == 1 else "slot"
+    tol = tol_for(dtype)
+    sl = seq_slices(P)
+    q, k, v = synth.prefill_qkv(w, 0, "cuda")
+    out = torch.empty_like(q)
+    st.prefill(0, q, k, v, out)
+    hk, hv = [], []
+    for b in range(B):
+        pos = np.arange(P[b])
+        qr, kr = oracle.rope(f64(q[sl[b]]), pos, theta), oracle.rope(f64(k[sl[b]]), pos, theta)
+        ref = oracle.prefill_window(qr, kr, f64(v[sl[b]]), w.scale, W)
+        assert np.max(np.abs(f64(out[sl[b]]) - ref)) <= tol, b
+        hk.append(list(kr))
+        hv.append(list(f64(v[sl[b]])))
+    for t in range(steps):
+        qs, kn, vn = synth.decode_qkv(w, 0, t, "cuda")
+        o = torch.empty_like(qs)
+        st.decode_step(0, qs, kn, vn, o)
+        for b in range(B):
+            p = [oracle.rope_position(pol, P[b], t, W)]
+            hk[b].append(oracle.rope(f64(kn[b])[None], p, theta)[0])
+            hv[b].append(f64(vn[b]))
+            K, V = np.stack(hk[b][-W:]), np.stack(hv[b][-W:])
+            qr = oracle.rope(f64(qs[b])[None], p, theta)[0]
+            for h in range(H):
+                ref = oracle.attend(qr[h], K[:, h], V[:, h], w.scale)
+                assert np.max(np.abs(f64(o[b, h]) - ref)) <= tol, (t, b, h)
+        st.advance()
+    assert st.check() == 0
