@@ -192,9 +192,9 @@ class DecodeRig:
         self.st = rswa.State(B, L, H, d, w.window, w.prefill_lens, dtype=w.dtype, n_generated=ng)
         if rope:
             self.st.set_rope(rope, 10000.0, stream=stream)
-        self.q = torch.empty(L, B, H, d, dtype=w.dtype, device="cuda")
-        self.kn = torch.empty_like(self.q)
-        self.vn = torch.empty_like(self.q)
+        # q, k_new, v_new of all layers in one buffer: one host copy per step
+        self.qkv = torch.empty(3, L, B, H, d, dtype=w.dtype, device="cuda")
+        self.q, self.kn, self.vn = self.qkv[0], self.qkv[1], self.qkv[2]
         self.out = torch.empty_like(self.q)
         for l in range(L):
             a, b_, c = synth.decode_qkv(w, l, 0, "cuda")
@@ -333,14 +333,12 @@ def e2e_tokens(rig: DecodeRig, steps: int, warmup: int, flush):
     outputs and the masked logits; all inside the timed region (the logits
     and history copies overlap the decode layers on a second stream)."""
     s = rig.s
-    hq = torch.empty(rig.q.shape, dtype=rig.q.dtype, pin_memory=True)
-    hk, hv = torch.empty_like(hq, pin_memory=True), torch.empty_like(hq, pin_memory=True)
-    hq.copy_(rig.q.cpu()); hk.copy_(rig.kn.cpu()); hv.copy_(rig.vn.cpu())
+    hqkv = rig.qkv.cpu().pin_memory()
     hl = rig.logits.cpu().pin_memory()
     hh = rig.hist.cpu().pin_memory()
-    ho = torch.empty_like(hq, pin_memory=True)
+    ho = torch.empty(rig.out.shape, dtype=rig.out.dtype, pin_memory=True)
     hlo = torch.empty_like(hl, pin_memory=True)
-    h2d = 3 * hq.numel() * hq.element_size() + hl.numel() * 4 + hh.numel() * 4
+    h2d = hqkv.numel() * hqkv.element_size() + hl.numel() * 4 + hh.numel() * 4
     d2h = ho.numel() * ho.element_size() + hlo.numel() * 4
 
     # The logits and histories are copied in on a second stream while the
@@ -348,7 +346,7 @@ def e2e_tokens(rig: DecodeRig, steps: int, warmup: int, flush):
     # starts after the step's start event, so it stays inside the timed region.
     from ring_sliding_window_b200 import rswa
     cs = torch.cuda.Stream()
-    ev_start, ev_in = torch.cuda.Event(), torch.cuda.Event()
+    ev_start, ev_in, ev_dec, ev_out = (torch.cuda.Event() for _ in range(4))
 
     def one():
         ev_start.record(s)
@@ -357,15 +355,19 @@ def e2e_tokens(rig: DecodeRig, steps: int, warmup: int, flush):
             rig.logits.copy_(hl, non_blocking=True)
             rig.hist.copy_(hh, non_blocking=True)
             ev_in.record(cs)
-        rig.q.copy_(hq, non_blocking=True)
-        rig.kn.copy_(hk, non_blocking=True)
-        rig.vn.copy_(hv, non_blocking=True)
+        rig.qkv.copy_(hqkv, non_blocking=True)
         rig.graph_dec.replay()
+        ev_dec.record(s)
+        # the outputs go back while the ban runs
+        cs.wait_event(ev_dec)
+        with torch.cuda.stream(cs):
+            ho.copy_(rig.out, non_blocking=True)
+            ev_out.record(cs)
         s.wait_event(ev_in)
         rswa.rswa_ngram_mask(rig.logits, rig.hist, None, synth.NGRAM_SIZE, synth.NGRAM_WINDOW,
                              stream=s)
-        ho.copy_(rig.out, non_blocking=True)
         hlo.copy_(rig.logits, non_blocking=True)
+        s.wait_event(ev_out)
 
     with torch.cuda.stream(s):
         for _ in range(warmup):
