@@ -59,25 +59,6 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define RSWA_EXP2_FMA_EVERY 0
 #endif
 constexpr int kEmuEvery = RSWA_EXP2_FMA_EVERY;
-// 1: P's exponentials in packed bf16 pairs (ex2.approx.ftz.bf16x2): the
-// argument x = s * scale*log2(e) - m is rounded to bf16 first (8-bit
-// mantissa), the result is the bf16 P the P V product reads anyway, and the
-// row sum adds the same rounded values.  Half the MUFU operations of the
-// fp32 path, but measured slower on B200 (804 vs 858 TFLOP/s multi-page),
-// so off by default.  Build-time knob: -DRSWA_EXP2_BF16X2=0|1.
-#ifndef RSWA_EXP2_BF16X2
-#define RSWA_EXP2_BF16X2 0
-#endif
-constexpr bool kExpBf16x2 = RSWA_EXP2_BF16X2 != 0;
-// 1: the two softmax warpgroups take turns on their exponential loops
-// (A(0), B(0), A(1), B(1), ...), keeping them half a period apart so each
-// has the MUFU pipe to itself while the tensor core runs the other tile's
-// MMAs.  Build-time knob: -DRSWA_SOFTMAX_ALTERNATE=0|1; off by default
-// because on B200 it measured slightly slower (830 vs 845 TFLOP/s, multi-page).
-#ifndef RSWA_SOFTMAX_ALTERNATE
-#define RSWA_SOFTMAX_ALTERNATE 0
-#endif
-constexpr bool kAlternate = RSWA_SOFTMAX_ALTERNATE != 0;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ constexpr uint32_t col_s(int x) { return (uint32_t)x * kTile; }        // 0, 128
@@ -95,7 +76,6 @@ struct __align__(1024) PrefillSmem {
   uint64_t o_bar[2];     // per query tile: one phase per finished PV_X
   uint64_t o_final[2];   // per query tile: the last PV_X finished
   uint64_t mma_done;     // everything the MMA thread issued finished
-  uint64_t exp_done[2];  // per query tile: its warpgroup finished tile j's exponentials
   uint32_t tmem_base;
   int dead;
 };
@@ -176,7 +156,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[x], 4);
       mbar_init(&sm.o_bar[x], 1);
       mbar_init(&sm.o_final[x], 1);
-      mbar_init(&sm.exp_done[x], 4);
     }
     mbar_init(&sm.mma_done, 1);
     sm.dead = 0;
@@ -339,12 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_use = m_new;
         alpha = tc::ex2(m_run - m_new);
       }
-      // take turns with the other warpgroup: A(j) after B(j-1), B(j) after A(j)
-      if (kAlternate && ntiles > 1) {
-        if (x == 0 && j > 0) ok = wait_bar(&sm.exp_done[1], (j - 1) & 1, v.err, dead);
-        if (x == 1 && j < n_kv_a) ok = wait_bar(&sm.exp_done[0], j & 1, v.err, dead);
-        if (!ok) break;
-      }
       uint64_t rs4[4];  // row sum as 4 packed pairs of partial sums
 #pragma unroll
       for (int i = 0; i < 4; ++i) rs4[i] = 0;
@@ -362,31 +335,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t xx = tc::ffma2(tc::f2_pack(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]),
                                         sl2x2, negm2);
           const float x0 = tc::f2_lo(xx), x1 = tc::f2_hi(xx);
-          if constexpr (kExpBf16x2) {
-            // both exponentials in one MUFU op, straight into the bf16 pair
-            // that P V consumes; the row sum adds exactly those values
-            const uint32_t pb = tc::ex2_bf16x2(tc::pack_bf16x2(x0, x1));
-            rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(__uint_as_float(pb << 16),
-                                                            __uint_as_float(pb & 0xffff0000u)));
-            pk[c] = pb;
-          } else {
-            // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
-            const bool emu =
-                kEmuEvery > 0 && (c % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
-            const float p0 = emu ? tc::exp2_fma(x0) : tc::ex2(x0);
-            const float p1 = emu ? tc::exp2_fma(x1) : tc::ex2(x1);
-            rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(p0, p1));
-            pk[c] = tc::pack_bf16x2(p0, p1);
-          }
+          // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
+          const bool emu = kEmuEvery > 0 && (c % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1;
+          const float p0 = emu ? tc::exp2_fma(x0) : tc::ex2(x0);
+          const float p1 = emu ? tc::exp2_fma(x1) : tc::ex2(x1);
+          rs4[c & 3] = tc::fadd2(rs4[c & 3], tc::f2_pack(p0, p1));
+          pk[c] = tc::pack_bf16x2(p0, p1);
         }
         tc::st32(t_s + 32 * half, pk);
       }
       const uint64_t r01 = tc::fadd2(tc::fadd2(rs4[0], rs4[1]), tc::fadd2(rs4[2], rs4[3]));
       const float rs = tc::f2_lo(r01) + tc::f2_hi(r01);
-      if (kAlternate && ntiles > 1) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.exp_done[x]);
-      }
       l_run = l_run * alpha + rs;
       m_run = m_use;
       if (j > 0 && rescale) {

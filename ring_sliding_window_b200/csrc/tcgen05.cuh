@@ -145,13 +145,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x for a packed pair of bf16 (one MUFU op for both), flush-to-zero.
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
 // 2^x on the FMA pipe, to take part of the softmax's exponentials off the
 // MUFU unit.  Range reduction x = j + f, j = rint(x) (read from the low
 // mantissa bits of x + 1.5 * 2^23), f in [-1/2, 1/2]; 2^f by the degree-3
