@@ -73,7 +73,6 @@ struct __align__(1024) PrefillSmem {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2];    // per query tile: S_X(j) finished
   uint64_t p_full[2];    // per query tile: P_X(j) written (4 warp arrivals)
-  uint64_t o_bar[2];     // per query tile: one phase per finished PV_X
   uint64_t o_final[2];   // per query tile: the last PV_X finished
   uint64_t mma_done;     // everything the MMA thread issued finished
   uint32_t tmem_base;
@@ -154,7 +153,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.s_full[x], 1);
       mbar_init(&sm.p_full[x], 4);
-      mbar_init(&sm.o_bar[x], 1);
       mbar_init(&sm.o_final[x], 1);
     }
     mbar_init(&sm.mma_done, 1);
@@ -243,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = wait_bar(&sm.p_full[x], j & 1, v.err, dead))) break;
           tc::fence_after_sync();
           issue_pv(tbase + col_o(x), tbase + col_s(x), smem_u32(sm.v[s]), j > 0);
-          tc::commit(&sm.o_bar[x]);
           if (j == nkv - 1) tc::commit(&sm.o_final[x]);
           // S_X(j+1) = Q_X K_{j+1}^T  (overwrites P_X(j): issued after PV_X(j))
           if (j + 1 < nkv) {
@@ -349,25 +346,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       l_run = l_run * alpha + rs;
       m_run = m_use;
       if (j > 0 && rescale) {
-        // O_X may only be touched once PV_X(j-1) has finished (S_X(j) was
-        // issued after it, so this wait normally returns at once)
-        ok = wait_bar(&sm.o_bar[x], (j - 1) & 1, v.err, dead);
-        if (ok) {
-          tc::fence_after_sync();
+        // O_X may only be touched once PV_X(j-1) has finished.  It has: the
+        // commit behind s_full (waited for above) tracks every MMA its thread
+        // issued before S_X(j), PV_X(j-1) included.
 #pragma unroll
-          for (int c4 = 0; c4 < kD / 32; ++c4) {
-            float o[32];
-            tc::ld32(t_o + 32 * c4, reinterpret_cast<uint32_t *>(o));
-            tc::wait_ld();
-            const uint64_t a2 = tc::f2_pack(alpha, alpha);
+        for (int c4 = 0; c4 < kD / 32; ++c4) {
+          float o[32];
+          tc::ld32(t_o + 32 * c4, reinterpret_cast<uint32_t *>(o));
+          tc::wait_ld();
+          const uint64_t a2 = tc::f2_pack(alpha, alpha);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const uint64_t r = tc::fmul2(tc::f2_pack(o[2 * c], o[2 * c + 1]), a2);
-              o[2 * c] = tc::f2_lo(r);
-              o[2 * c + 1] = tc::f2_hi(r);
-            }
-            tc::st32(t_o + 32 * c4, reinterpret_cast<const uint32_t *>(o));
+          for (int c = 0; c < 16; ++c) {
+            const uint64_t r = tc::fmul2(tc::f2_pack(o[2 * c], o[2 * c + 1]), a2);
+            o[2 * c] = tc::f2_lo(r);
+            o[2 * c + 1] = tc::f2_hi(r);
           }
+          tc::st32(t_o + 32 * c4, reinterpret_cast<const uint32_t *>(o));
         }
       }
       tc::wait_st();
