@@ -266,6 +266,18 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
       ++pre_stages;
     }
   }
+  // The first piece's q, k_new and v_new rows and its ring counter are read
+  // right after the wait: start their trip to L2 now (a prefetch returns no
+  // value, so a row still being written by an earlier kernel is read fresh).
+  if (warp == 0 && lane < 7) {
+    const int64_t in_off = ((int64_t)first_piece.b * v.H + first_piece.h) * D;
+    const uint8_t *row = lane < 2 ? (const uint8_t *)a.q
+                       : lane < 4 ? (const uint8_t *)a.k_new : (const uint8_t *)a.v_new;
+    if (lane < 6)
+      prefetch_l2(row + in_off * (int64_t)sizeof(T) + (lane & 1) * (D * sizeof(T) / 2));
+    else
+      prefetch_l2(v.t + first_piece.b);
+  }
   // From here on the kernel reads q/k_new/v_new, the ring counters and ring
   // rows of the cache, which earlier kernels in the stream may still be
   // producing.

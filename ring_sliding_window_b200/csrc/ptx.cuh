@@ -115,6 +115,13 @@ __device__ __forceinline__ void allow_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Pull the line holding p into L2.  A hint with no value returned: a later
+// write by another kernel lands in the same coherent L2, so it may be issued
+// before the grid-dependency wait for data that is still being produced.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ------------------------------------------------------------- clusters
 // Shared-memory address of `p` (a variable of this CTA) in the CTA of the
 // cluster with rank `rank`.
