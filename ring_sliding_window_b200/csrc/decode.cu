@@ -500,16 +500,33 @@ __global__ void __launch_bounds__(DecodeShape<T, D>::kThreads)
       cluster_arrive_release();
       cluster_wait_acquire();
       if (rank == 0 && tid < D) {
+        // unrolled to the largest cluster, so all C partials' loads and
+        // exponentials are in flight together (a loop to the run-time C was
+        // two dependent chains of C shared-memory loads)
         const int C = v.cluster_size;
-        float Mg = -INFINITY;
-        for (int r = 0; r < C; ++r) Mg = fmaxf(Mg, sm.cl_ml[r].x);
+        float2 ml[kMaxCluster];
+        float ov[kMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r) {
+          ml[r] = r < C ? sm.cl_ml[r] : make_float2(-INFINITY, 0.f);
+          ov[r] = r < C ? sm.cl_o[r][tid] : 0.f;
+        }
+        float mx[4] = {ml[0].x, ml[1].x, ml[2].x, ml[3].x};
+#pragma unroll
+        for (int r = 4; r < kMaxCluster; ++r) mx[r & 3] = fmaxf(mx[r & 3], ml[r].x);
+        const float Mg = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         float Lg = 0.f, acc = 0.f;
-        if (Mg != -INFINITY)
-          for (int r = 0; r < C; ++r) {
-            const float wgt = exp2f(sm.cl_ml[r].x - Mg);  // 0 for an empty range
-            Lg = fmaf(wgt, sm.cl_ml[r].y, Lg);
-            acc = fmaf(wgt, sm.cl_o[r][tid], acc);
+        if (Mg != -INFINITY) {
+          float l4[4] = {0.f, 0.f, 0.f, 0.f}, a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r) {
+            const float wgt = exp2f(ml[r].x - Mg);  // 0 for an empty range or an absent rank
+            l4[r & 3] = fmaf(wgt, ml[r].y, l4[r & 3]);
+            a4[r & 3] = fmaf(wgt, ov[r], a4[r & 3]);
           }
+          Lg = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+          acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        }
         store_result<T, D>(v, a, pc.b * v.H + pc.h, tid, Mg, Lg, acc);
       }
       continue;  // a cluster CTA has exactly one piece
