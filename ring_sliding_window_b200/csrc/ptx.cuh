@@ -88,6 +88,12 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
+// Ask the TMA unit to pull [p, p + bytes) into L2: no destination, nothing to
+// wait for.  p 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // 4-byte asynchronous global -> shared copy (no register staging); complete
 // with cp_async_wait_all() and a barrier before the data is read.
 __device__ __forceinline__ void cp_async_4(void *smem_dst, const void *src) {

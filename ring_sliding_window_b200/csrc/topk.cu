@@ -141,7 +141,9 @@ __device__ void reject_row(const TopkArgs &a, int row, int rank) {
 }
 
 // The streaming pass shared by both kernels: each thread reads its 64 columns
-// once (two batches of four 16-byte loads in flight) and keeps the two first
+// once (two batches of four 16-byte loads in flight; in the top-1 form the
+// CTA's whole range is first requested into L2 by bulk prefetches, so the
+// row streams from DRAM at full depth) and keeps the two first
 // maxima of them in increasing column order; the ban is worked out while the
 // last two batches are in flight (the history was copied asynchronously at
 // the start).  If a thread's best is banned its second is the answer, unless
@@ -156,6 +158,18 @@ __device__ __forceinline__ unsigned long long stream_thread_max(const TopkArgs &
                                                                 int32_t *hist_s, int *bad) {
   const int tid = threadIdx.x;
   const float *lrow = a.logits + (int64_t)row * a.ld;
+  if (kEvictFirst) {
+    // single-pass (top-1) form: the CTA's whole column range on its way into
+    // L2 at once (the loads below keep only two batches per thread in
+    // flight).  The row and col0 are 16-byte aligned, and col0 < vocab.
+    // (The two-pass top-k form measured slower with it.)
+    const int ncols = min(kChunk, a.vocab - col0);
+    const uint32_t bytes = (uint32_t)(ncols * 4) & ~15u;
+    constexpr uint32_t kPiece = 4096;
+    for (uint32_t off = (uint32_t)tid * kPiece; off < bytes; off += kThreads * kPiece)
+      bulk_prefetch_l2(reinterpret_cast<const char *>(lrow + col0) + off,
+                       bytes - off < kPiece ? bytes - off : kPiece);
+  }
   stage_history(a, row, hist_s);
   constexpr int kBatch = 4;
   static_assert(kF4PerThread == 4 * kBatch, "four batches per thread");
