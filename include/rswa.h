@@ -403,7 +403,7 @@ const char *rswa_status_string(rswa_status status);
 const char *rswa_last_cuda_error(void);
 
 /* ---- Allocation-free decode step --------------------------------------
- * This call has no counterpart in the paper; it exists for callers that
+ * This call has no counterpart in the method itself; it exists for callers that
  * cannot hand the library a workspace.  A plugin hosted by another runtime
  * or inference server gets its input and output tensors but may not allocate
  * device memory itself (the host application's allocator owns the pool, so a
