@@ -215,21 +215,39 @@ class DecodeRig:
         self.graph = None
 
     def prefill_all(self, flush, time_it=True):
-        """Run rswa_prefill on every layer; returns per-layer event times (ms)."""
+        """Run rswa_prefill on every layer (this fills the caches); then time
+        each layer's call replayed from a CUDA graph after an L2 flush, so the
+        host side of the call (argument checks, tensor-map encoding, Python
+        marshalling) stays outside the events and the inputs are cold.
+        Returns per-layer event times (ms)."""
         w = self.w
         q, k, v = synth.prefill_qkv(w, 0, "cuda")
         out = torch.empty_like(q)
-        times = []
         with torch.cuda.stream(self.s):
             for l in range(w.layers):
+                self.st.prefill(l, q, k, v, out, stream=self.s)
+        self.s.synchronize()
+        if not time_it:
+            return []
+        graphs = []
+        for l in range(w.layers):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.s):
+                self.st.prefill(l, q, k, v, out, stream=self.s)
+            graphs.append(g)
+        times = []
+        with torch.cuda.stream(self.s):
+            for g in graphs:
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(self.s)
-                self.st.prefill(l, q, k, v, out, stream=self.s)
+                g.replay()
                 e1.record(self.s)
                 times.append((e0, e1))
         self.s.synchronize()
-        return [a.elapsed_time(b) for a, b in times]
+        res = [a.elapsed_time(b) for a, b in times]
+        del graphs
+        return res
 
     def token(self):
         from ring_sliding_window_b200 import rswa

@@ -445,9 +445,16 @@ cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k,
   if (!make_tmap(&tq, q, v.total_tokens, v.H) || !k_ok || !make_tmap(&tv, vv, v.total_tokens, v.H))
     return cudaErrorInvalidValue;
   const int smem = (int)sizeof(PrefillSmem) + 1024;
-  cudaError_t e =
-      cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // the attribute holds per device for the life of the process: set it once
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   PrefillTcArgs args{v, blocks, (__nv_bfloat16 *)out, kc ? 1 : 0};
   prefill_tc_kernel<<<n_blocks, kThreads, smem, s>>>(tq, tk, tv, args);
   return cudaGetLastError();
