@@ -304,7 +304,10 @@ rswa_status rswa_prefill(rswa_state *state, int32_t layer, const void *q, const 
  * dependents start early (griddepcontrol.launch_dependents), and it then
  * reads prompt rows (slots < P_b) of this layer's cache before waiting for
  * that kernel.  A kernel that writes prompt rows must therefore not release
- * its dependents early; everything else is read after the wait.
+ * its dependents early; everything else is read after the wait.  (Before the
+ * wait it also asks L2 for the lines of q, k_new, v_new and t_b: a prefetch
+ * returns nothing, so rows an earlier kernel is still writing are read fresh
+ * after the wait.)
  * RSWA_ESTATE if the layer was never prefilled. */
 rswa_status rswa_decode_step(rswa_state *state, int32_t layer, const void *q, const void *k_new,
                              const void *v_new, void *out, void *stream);
