@@ -151,11 +151,15 @@ __device__ void reject_row(const TopkArgs &a, int row, int rank) {
 // skipping banned ones -- which needs two banned tokens among one thread's 64
 // columns.  Returns the thread's largest masked key ((order image of the
 // masked value) << 32 | ~column), 0 if it has no column, and sets *bad to
-// the row's error bits (the same in every CTA of the row).
+// the row's error bits (the same in every CTA of the row).  With `second`,
+// also its second largest masked key where the two tracked maxima give it
+// exactly (neither banned, the second finite), else kKeyUnknown.
+constexpr unsigned long long kKeyUnknown = ~0ull;  // above every real key
 template <bool kEvictFirst>
 __device__ __forceinline__ unsigned long long stream_thread_max(const TopkArgs &a, int row,
                                                                 int col0, uint32_t *ban_bits,
-                                                                int32_t *hist_s, int *bad) {
+                                                                int32_t *hist_s, int *bad,
+                                                                unsigned long long *second = nullptr) {
   const int tid = threadIdx.x;
   const float *lrow = a.logits + (int64_t)row * a.ld;
   if (kEvictFirst) {
@@ -227,6 +231,10 @@ __device__ __forceinline__ unsigned long long stream_thread_max(const TopkArgs &
     const int f = col - col0;
     return ((ban_bits[f >> 5] >> (f & 31)) & 1u) != 0;
   };
+  if (second)
+    *second = (b1 != -INFINITY && !banned(i1) && b2 != -INFINITY && !banned(i2) && i2 < a.vocab)
+                  ? ((unsigned long long)ord_fast(b2) << 32) | (0xFFFFFFFFu - (uint32_t)i2)
+                  : kKeyUnknown;
   float best = b1;
   int bi = i1;
   if (b1 != -INFINITY && banned(i1)) {
@@ -397,7 +405,9 @@ __global__ void __launch_bounds__(kThreads, 4)
     n_top = 0;
   }
   int bad = 0;
-  const unsigned long long key = stream_thread_max<false>(a, row, col0, ban_bits, hist_s, &bad);
+  unsigned long long key2;
+  const unsigned long long key = stream_thread_max<false>(a, row, col0, ban_bits, hist_s, &bad,
+                                                          &key2);
   if (bad) {  // the same in every CTA of the row
     if (rank == 0 && tid == 0 && a.err) atomicOr(a.err, bad);
     reject_row(a, row, rank);
@@ -415,12 +425,21 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
   cluster_arrive_release();
   cluster_wait_acquire();
-  // ---- 3. this CTA's keys >= T to the leader (its key buffer is free again)
+  // ---- 3. this CTA's keys >= T to the leader (its key buffer is free again).
+  // A thread whose largest key is below T has none; one whose second largest
+  // is known and below T has only its largest; any other thread with a key
+  // >= T rereads its columns (from L2).
   {
     const unsigned long long T = thr;
     const uint32_t cand_addr = map_to_rank(keybuf, 0);
     const uint32_t count_addr = map_to_rank(&n_cand, 0);
-    for (int i0 = 0; i0 < kF4PerThread; i0 += 8) {
+    const bool only_first = key >= T && key2 < T;
+    if (only_first) {
+      const uint32_t slot = atom_add_cluster_u32(count_addr, 1u);
+      if (slot < (uint32_t)kTopkCandidates) st_cluster_u64(cand_addr + 8u * slot, key);
+    }
+    const bool reread = key >= T && !only_first;
+    for (int i0 = 0; reread && i0 < kF4PerThread; i0 += 8) {
       float4 y[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -451,25 +470,38 @@ __global__ void __launch_bounds__(kThreads, 4)
   cluster_wait_acquire();
   if (rank != 0) return;  // the leader reads only its own shared memory from here
 
-  // ---- 4. the k largest candidates, ordered
+  // ---- 4. the k largest candidates, ordered.  Keys are distinct (they hold
+  // the column).  Up to one candidate per thread: each counts the larger
+  // ones, its rank, and the k first ranks are the answer in order.  More:
+  // a radix select of the k-th largest, then the same ranking among those.
   const int k = a.k;
   const int nc = min((int)n_cand, kTopkCandidates);
-  const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel);
-  for (int i = tid; i < nc; i += kThreads) {
-    const unsigned long long kk = keybuf[i];
-    if (kk >= T2) {
-      const uint32_t slot = atomicAdd(&n_top, 1u);
-      if (slot < (uint32_t)kTopkMax) top[slot] = kk;
+  if (nc <= kThreads) {
+    if (tid < nc) {
+      const unsigned long long mine = keybuf[tid];
+      int r = 0;
+      for (int j = 0; j < nc; ++j) r += keybuf[j] > mine;
+      if (r < k) sorted[r] = mine;
     }
+    __syncthreads();
+  } else {
+    const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel);
+    for (int i = tid; i < nc; i += kThreads) {
+      const unsigned long long kk = keybuf[i];
+      if (kk >= T2) {
+        const uint32_t slot = atomicAdd(&n_top, 1u);
+        if (slot < (uint32_t)kTopkMax) top[slot] = kk;
+      }
+    }
+    __syncthreads();
+    if (tid < k) {
+      const unsigned long long mine = top[tid];
+      int r = 0;
+      for (int j = 0; j < k; ++j) r += top[j] > mine;
+      sorted[r] = mine;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  if (tid < k) {
-    const unsigned long long mine = top[tid];
-    int r = 0;
-    for (int j = 0; j < k; ++j) r += top[j] > mine;
-    sorted[r] = mine;
-  }
-  __syncthreads();
   if (tid < k) {
     const unsigned long long kk = sorted[tid];
     const int col = (int)(0xFFFFFFFFu - (uint32_t)kk);
