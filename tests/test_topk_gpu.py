@@ -221,3 +221,29 @@ def test_topk_two_banned_in_one_thread_and_banned_lone_maximum(k):
                         _two_ban_history(window, n, [7], vocab, 3)])
     idx = _check(logits, hist, None, n, window, k, False)
     assert idx[0, 0] not in (1000, 2024) and idx[1, 0] == 0 and idx[2, 0] == 1000
+
+
+@pytest.mark.parametrize("tied", [False, True], ids=["distinct", "tied"])
+def test_topk_many_candidates_in_few_threads(tied):
+    """More than 256 candidates reach the leader (the radix-select branch of
+    the final selection), and threads hold more than two keys >= T (the
+    reread branch): every column of five threads' strided ranges (thread t of
+    the CTA at column offset 16,384 rho reads columns
+    16,384 rho + 4 (t + 256 i) + u, i < 16, u < 4) gets a value far above the
+    rest, so the threshold from the thread maxima lets 320 of them through."""
+    rows, k = 3, 64
+    logits, hist, _ = synth.ngram_inputs(rows, synth.VOCAB, synth.NGRAM_SIZE, synth.NGRAM_WINDOW,
+                                         synth.seed(5, 0, 900_000 + int(tied)))
+    cols = []
+    for rho, t in ((1, 0), (1, 37), (2, 100), (5, 200), (7, 255)):
+        for i in range(16):
+            for u in range(4):
+                c = 16384 * rho + 4 * (t + 256 * i) + u
+                if c < synth.VOCAB:
+                    cols.append(c)
+    cols = torch.tensor(cols)
+    planted = torch.full((len(cols),), 50.0) if tied else 50.0 + 0.001 * torch.arange(len(cols))
+    logits[:, cols] = planted
+    idx = _check(logits, hist, None, synth.NGRAM_SIZE, synth.NGRAM_WINDOW, k, False)
+    # the k chosen are planted columns (a banned follower may have taken one out)
+    assert np.isin(idx, cols.numpy()).all()
