@@ -96,3 +96,13 @@ def test_reference_arm_line_carries_the_contract_fields():
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_bench_rejects_fewer_than_three_warmup_steps():
+    """The timing rules ask for at least 3 untimed warm-up steps."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "2"], capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode != 0
+    assert "--warmup must be >= 3" in r.stderr
+    assert r.stdout.strip() == ""
