@@ -95,3 +95,36 @@ def test_null_state_and_ngram_args_rejected(rswa):
     assert lib.rswa_ngram_mask(None, 10, 4096, 4, None, 1, 10, 2, 4, None, None) == rswa.RSWA_EINVAL
     # zero rows: valid no-op, nothing launched
     assert lib.rswa_ngram_mask(None, 10, None, 4, None, 0, 10, 2, 4, None, None) == rswa.RSWA_OK
+
+
+def test_topk_combine_and_setter_args_rejected(rswa):
+    """The later entry points check their arguments on the host and return
+    RSWA_EINVAL before any launch (or RSWA_OK for an empty call)."""
+    lib = rswa.lib
+    E, OK = rswa.RSWA_EINVAL, rswa.RSWA_OK
+    A = 4096  # a 16-byte-aligned stand-in address: never dereferenced on these paths
+
+    def topk(logits=A, ld=16, hist=A, hist_ld=4, rows=1, vocab=16, n=2, window=4, k=2,
+             uniform=None, temperature=1.0, top_idx=A):
+        return lib.rswa_ngram_topk(logits, ld, hist, hist_ld, None, rows, vocab, n, window, k, 0,
+                                   uniform, temperature, top_idx, None, None, None, None)
+
+    for kw in (dict(rows=-1), dict(vocab=0), dict(vocab=rswa.RSWA_TOPK_MAX_VOCAB + 1, ld=1 << 20),
+               dict(n=0), dict(window=-1), dict(k=0), dict(k=rswa.RSWA_TOPK_MAX + 1, vocab=128, ld=128),
+               dict(k=17), dict(ld=15), dict(ld=18), dict(hist_ld=3), dict(window=8193, hist_ld=8193),
+               dict(uniform=A, temperature=0.0), dict(uniform=A, temperature=float("inf")),
+               dict(logits=None), dict(logits=A + 4), dict(top_idx=None), dict(hist=None)):
+        assert topk(**kw) == E, kw
+    assert topk(rows=0, logits=None, top_idx=None) == OK  # empty: nothing launched
+
+    def combine(ml=A, o=A, shares=2, rings=3, d=128, dtype=rswa.RSWA_BF16, out=A):
+        return lib.rswa_combine_partials(ml, o, shares, rings, d, dtype, out, None)
+
+    for kw in (dict(shares=0), dict(rings=-1), dict(d=96), dict(dtype=7), dict(ml=None),
+               dict(o=None), dict(out=None)):
+        assert combine(**kw) == E, kw
+    assert combine(rings=0, ml=None, o=None, out=None) == OK
+
+    assert lib.rswa_state_set_rope(None, 1, 10000.0, None) == E
+    assert lib.rswa_state_set_attention(None, 1) == E
+    assert lib.rswa_decode_step_partial(None, 0, A, A, A, 0, 10, A, A, None) == E
