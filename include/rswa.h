@@ -430,13 +430,21 @@ const char *rswa_last_cuda_error(void);
  * every device that loads the library, held until the process exits.  The
  * call allocates nothing (no cudaMalloc/cudaFree).  Its first call on a
  * device looks up the array's device address (cudaGetSymbolAddress); make
- * that first call before any stream capture.  The work tables are copied into
- * the array from pageable host memory on `stream` at every call.  Every call
- * on a device shares the one array and it keeps the last call's contents, so
- * calls whose work overlaps on the GPU (different streams, no ordering)
- * race and corrupt each other; order them on one stream.
+ * that first call before any stream capture.  At every call the work tables
+ * are written into the array by small kernels enqueued on `stream` that carry
+ * the bytes in their launch parameters, so no host memory is referenced once
+ * the call has returned.  Every call on a device shares the one array and it
+ * keeps the last call's contents, so calls whose work overlaps on the GPU
+ * (different streams, no ordering) race and corrupt each other; order them
+ * on one stream.
  * Returns RSWA_EINVAL for bad arguments and RSWA_ENOMEM when the batch needs
- * more scratch than the array holds (rswa_workspace_bytes() > the limit). */
+ * more scratch than the array holds.  What counts is the decode step's part of
+ * a workspace: error word, ring counters, P_b, slot bases, the split-K work
+ * tables and the partials.  The keys of all rings are cut into one range per
+ * decode CTA (3 per SM), so there are at most (CTAs + B*H) pieces, each
+ * taking 32 bytes of table and 8 + 4d bytes of partials: about 0.6 MiB for
+ * 64 requests of 10 heads at d = 128 on a 148-SM part, whatever the prompt
+ * lengths; about 7,000 (b, h) rings of d = 128 fit. */
 #define RSWA_NOALLOC_SCRATCH_BYTES (4u << 20)
 rswa_status rswa_decode_step_noalloc(const rswa_config *cfg, const int64_t *prefill_len,
                                      const int64_t *n_generated, void *k_cache, void *v_cache,

@@ -18,6 +18,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -52,6 +53,49 @@ rswa_status scratch_for_device(int dev, uint8_t **out) {
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Sections of the array that the decode kernel reads or writes, in the
+// workspace's order.  Only these count against the limit: the prefill and
+// RoPE tables of a full workspace are never touched by a decode step.
+struct NoAllocLayout {
+  size_t err, t, plen, slot_base, pieces, cta_piece, bh_piece, bh_count, part_ml, part_o, total;
+};
+
+NoAllocLayout noalloc_layout(const rswa_config *c, const DecodePlan &p) {
+  const size_t B = (size_t)c->batch, BH = B * (size_t)c->num_heads;
+  NoAllocLayout w;
+  size_t off = 0;
+  w.err = off;       off = align256(off + 2 * sizeof(int32_t));  // error word, fault flags
+  w.t = off;         off = align256(off + 2 * B * sizeof(int64_t));
+  w.plen = off;      off = align256(off + B * sizeof(int32_t));
+  w.slot_base = off; off = align256(off + (B + 1) * sizeof(int64_t));
+  w.pieces = off;    off = align256(off + (size_t)p.n_pieces * sizeof(DecodePiece));
+  w.cta_piece = off; off = align256(off + ((size_t)p.grid + 1) * sizeof(int32_t));
+  w.bh_piece = off;  off = align256(off + (BH + 1) * sizeof(int32_t));
+  w.bh_count = off;  off = align256(off + BH * sizeof(int32_t));
+  w.part_ml = off;   off = align256(off + (size_t)p.n_pieces * sizeof(float2));
+  w.part_o = off;    off = align256(off + (size_t)p.n_pieces * c->head_dim * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+// The work tables travel to the array inside kernel parameters: the launch
+// copies its parameters when it is enqueued, so nothing refers to the
+// caller's (or this call's) host memory once the call has returned.
+constexpr int kUploadChunk = 16384;
+struct __align__(16) UploadChunk {
+  uint8_t bytes[kUploadChunk];
+};
+
+__global__ void __launch_bounds__(256) noalloc_upload_kernel(uint8_t *dst,
+                                                             const __grid_constant__ UploadChunk c,
+                                                             int n16) {
+  const uint4 *src = reinterpret_cast<const uint4 *>(c.bytes);
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+  for (int i = threadIdx.x; i < n16; i += blockDim.x) d[i] = src[i];
+}
+
 }  // namespace
 }  // namespace rswa
 
@@ -76,7 +120,7 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
 
   const DecodePlan plan =
       plan_decode(cfg, prefill_len, nullptr, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
-  const WsLayout ws = layout_ws(cfg, prefill_len, plan);
+  const NoAllocLayout ws = noalloc_layout(cfg, plan);
   if (ws.total > kNoAllocScratchBytes) return RSWA_ENOMEM;  // batch too large for the array
 
   uint8_t *scratch = nullptr;
@@ -86,6 +130,8 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
   // Host image of the tables.  The error word and the per-(b, h) completion
   // counters in it are zero, so every call starts from cleared values; the
   // partials are fully overwritten by the split kernel and need no clearing.
+  // part_ml is 256-byte aligned, so the image is a whole number of 16-byte
+  // words.
   std::vector<uint8_t> img(ws.part_ml, 0);
   int64_t *t = (int64_t *)(img.data() + ws.t);
   int32_t *pl = (int32_t *)(img.data() + ws.plen);
@@ -100,10 +146,13 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
   memcpy(img.data() + ws.cta_piece, plan.cta_piece.data(), plan.cta_piece.size() * sizeof(int32_t));
   memcpy(img.data() + ws.bh_piece, plan.bh_piece.data(), plan.bh_piece.size() * sizeof(int32_t));
   cudaStream_t s = (cudaStream_t)stream;
-  // Pageable source: the call returns once the bytes are staged, so `img`
-  // may go out of scope; the copy is ordered before the kernels on `s`.
-  if (cudaMemcpyAsync(scratch, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return RSWA_ECUDA;
+  UploadChunk chunk;
+  for (size_t off = 0; off < img.size(); off += kUploadChunk) {
+    const size_t n = std::min(img.size() - off, (size_t)kUploadChunk);
+    memcpy(chunk.bytes, img.data() + off, n);
+    noalloc_upload_kernel<<<1, 256, 0, s>>>(scratch + off, chunk, (int)(n / 16));
+    if (cudaGetLastError() != cudaSuccess) return RSWA_ECUDA;
+  }
 
   DeviceView v;
   memset(&v, 0, sizeof(v));
@@ -128,8 +177,8 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
   v.part_o = (float *)(scratch + ws.part_o);
   v.decode_grid = plan.grid;
   v.n_pieces = plan.n_pieces;
-  // Plain launch (no programmatic dependent launch): the table upload just
-  // before it must be complete when the kernel starts.
+  // Plain launch (no programmatic dependent launch): the table upload
+  // kernels just before it must be complete when it starts.
   return launch_decode(v, q, k_new, v_new, k_cache, v_cache, out, s, false) == cudaSuccess
              ? RSWA_OK
              : RSWA_ECUDA;
