@@ -7,30 +7,33 @@
 // from the masked scores.  Selection follows a total order: larger masked
 // value first, the lower column first among equal values; NaN ranks as -inf.
 //
-// Design (HBM-bound: each logit is read once):
+// Design (HBM-bound: each logit is read once from DRAM):
 //  - One thread-block cluster of C = ceil(vocab / 16384) CTAs per row; each
-//    CTA holds its 16,384 columns in registers (64 per thread, 16 float4
-//    loads in flight per thread), so the row is read from HBM exactly once.
-//  - The ban: the row's history is staged in shared memory and every thread
-//    tests one candidate start of the windowed n-gram match at a time; the
-//    banned tokens in this CTA's columns are marked in a shared-memory
-//    bitmap (and, on request, -inf is stored over them in the logits).
+//    CTA streams its 16,384 columns (64 per thread, in four batches of four
+//    16-byte loads, two batches in flight) and keeps, per thread, the first
+//    two maxima of its columns in increasing column order.
+//  - The ban: the row's history is copied to shared memory asynchronously at
+//    kernel start and worked out while the last batches are in flight; every
+//    thread tests candidate starts of the windowed n-gram match; the banned
+//    tokens in this CTA's columns go into a shared-memory bitmap (and, on
+//    request, -inf is stored over them in the logits).  A thread whose best
+//    column is banned falls back on its second, and rescans its columns
+//    (from L2) only if both are banned.
 //  - Every column gets a 64-bit key: the order-preserving image of its masked
 //    value in the high word, (2^32 - 1 - column) in the low word, so keys
 //    are distinct and "larger key" is exactly the selection order.
-//  - k = 1 (its own kernel, nothing held): each thread streams its columns
-//    in increasing order keeping the first strict maximum, which costs one
-//    compare and two selects per column; the bitmap is consulted only when
-//    the maximum would change.  The (value, column) maxima are reduced over
-//    the warp, the CTA and, through distributed shared memory, the cluster.
-//    Few registers and little shared memory: the whole grid is one wave.
-//  - k > 1: radix select, 8 bits at a time from the top: each CTA histograms
-//    the digit of the keys that still match the chosen prefix, every CTA
-//    reads all CTAs' histograms through distributed shared memory and picks
-//    the digit holding the k-th largest key; this stops as soon as that
-//    digit's bin holds exactly the keys still needed (at the latest after
-//    the 8th digit, keys being distinct).  The keys at or above the final
-//    prefix -- exactly k -- go to the leader, which orders them.
+//  - k = 1 (its own kernel): the thread maxima are reduced over the warp, the
+//    CTA and, through distributed shared memory, the cluster's leader.  The
+//    CTA's column range is requested into L2 by bulk prefetches at kernel
+//    start, so the row leaves DRAM at full depth.
+//  - k > 1: the leader gathers the C x 256 thread maxima and finds their k-th
+//    largest, T, by a CTA-local radix select (8 bits per pass).  At least k
+//    keys of the row are >= T, and they all lie in the k threads whose
+//    maximum is >= T.  A thread whose second largest key is known and below T
+//    sends only its maximum; the others with a maximum >= T reread their
+//    columns (from L2) and send every key >= T.  The leader ranks up to 256
+//    candidates directly (each thread counts the larger ones), else first
+//    radix-selects the k-th largest among them.
 //  - Sampling: p_i proportional to exp((x_i - x_0) / T) over the k survivors
 //    (x_0 the largest), inverse CDF at the caller's uniform u in [0, 1).
 #include <cuda_runtime.h>
