@@ -315,6 +315,16 @@ def timed_tokens(rig: DecodeRig, steps: int, warmup: int, flush, sampler=None):
     return ms, ts, clocks
 
 
+def fill_ring(rig: DecodeRig):
+    """Replay the token graph until every ring holds W generated entries (the
+    method's warm-up phase); untimed."""
+    need = rig.w.window - min(rig.ring_t())
+    with torch.cuda.stream(rig.s):
+        for _ in range(max(0, need)):
+            rig.graph.replay()
+    rig.s.synchronize()
+
+
 def timed_decode_launches(rig: DecodeRig, reps: int, flush):
     """Average duration of one decode_split_kernel launch (one rswa_decode_step)
     in the bench's launch configuration: a CUDA graph of the layers' decode
@@ -408,34 +418,100 @@ def e2e_tokens(rig: DecodeRig, steps: int, warmup: int, flush):
 
 
 # --------------------------------------------------------------------------
-def cpu_oracle_rate(w: synth.Workload, seconds: float, max_steps=None, layers_per_step=None):
-    """The oracle as it stands, on this host's cores: decode steps (all layers of
-    the batch, plus the n-gram ban) from t = 0 until `seconds` have passed."""
-    import numpy as np
+def host_cpu():
+    """(logical CPUs this process may use, CPU model name) of this host."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 0
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    return n, model
 
+
+class OracleSample:
+    """The oracle as it stands, on this host's cores, over a bounded sample of
+    a workload: `layers` layers of the sequences `seqs`, each with every head,
+    prefilled with N(0,1) keys and values, then decoded from t = 0.  A step
+    runs the sampled layers' ring steps and the n-gram ban of the whole batch
+    (n = 35, window = 128).  The attention part is scaled to the whole model by
+    its key count (sampled keys / all keys of all layers), the ban is counted
+    once per step, so `rate()` is full-model decode steps per second."""
+
+    def __init__(self, w: synth.Workload, layers: int, seqs):
+        import numpy as np
+
+        import oracle
+        self.w, self.layers, self.seqs = w, layers, list(seqs)
+        rng = np.random.default_rng(0)
+        plens = [w.prefill_lens[b] for b in self.seqs]
+        self.model = oracle.RingModel(plens, w.window, layers, w.heads, w.head_dim)
+        for l in range(layers):
+            for i, P in enumerate(plens):
+                self.model.prefill(l, i, rng.standard_normal((P, w.heads, w.head_dim)),
+                                   rng.standard_normal((P, w.heads, w.head_dim)))
+        nb = len(plens)
+        self.qkv = [rng.standard_normal((3, nb, w.heads, w.head_dim)) for _ in range(layers)]
+        logits, hist, _ = synth.ngram_inputs(w.batch, synth.VOCAB, synth.NGRAM_SIZE,
+                                             synth.NGRAM_WINDOW, 1)
+        self.lg, self.hi = logits.numpy(), hist.numpy()
+        keys = lambda ps: sum(P + w.window for P in ps)  # noqa: E731 (steady-state keys)
+        self.fraction = layers * keys(plens) / (w.layers * keys(w.prefill_lens))
+        self.steps, self.attn_s, self.ban_s = 0, 0.0, 0.0
+
+    def run(self, seconds: float = 0.0, max_steps=None):
+        import oracle
+        w = self.w
+        t_start = time.perf_counter()
+        n = 0
+        while True:
+            t0 = time.perf_counter()
+            for l in range(self.layers):
+                q, kn, vn = self.qkv[l]
+                self.model.step(l, q, kn, vn, w.scale)
+            t1 = time.perf_counter()
+            oracle.ngram_ban(self.lg, self.hi, None, synth.NGRAM_SIZE, synth.NGRAM_WINDOW)
+            t2 = time.perf_counter()
+            self.attn_s += t1 - t0
+            self.ban_s += t2 - t1
+            self.steps += 1
+            n += 1
+            if max_steps is not None and n >= max_steps:
+                break
+            if max_steps is None and time.perf_counter() - t_start >= seconds and n >= 2:
+                break
+        return n
+
+    def reset_timers(self):
+        self.steps, self.attn_s, self.ban_s = 0, 0.0, 0.0
+
+    def rate(self) -> float:
+        per_step = self.attn_s / self.steps / self.fraction + self.ban_s / self.steps
+        return 1.0 / per_step
+
+    def describe(self) -> str:
+        w = self.w
+        return (f"{self.steps} decode steps of {self.layers} of {w.layers} layers x "
+                f"{len(self.seqs)} of {w.batch} sequences (all {w.heads} heads) of {w.name} "
+                f"from t = 0, plus the n-gram ban of the batch; {self.attn_s + self.ban_s:.1f} s. "
+                f"Attention scaled to the whole model by its key count "
+                f"(sample = {self.fraction:.4f} of the keys); the first W steps attend over "
+                f"fewer keys than steady state ({w.window} of "
+                f"{min(w.prefill_lens) + w.window} at most)")
+
+
+def cpu_baseline_block(sample: OracleSample) -> dict:
     import oracle
-    L = w.layers if layers_per_step is None else layers_per_step
-    rng = np.random.default_rng(0)
-    model = oracle.RingModel(w.prefill_lens, w.window, L, w.heads, w.head_dim)
-    for l in range(L):
-        for b, P in enumerate(w.prefill_lens):
-            model.prefill(l, b, rng.standard_normal((P, w.heads, w.head_dim)),
-                          rng.standard_normal((P, w.heads, w.head_dim)))
-    qkv = [rng.standard_normal((3, w.batch, w.heads, w.head_dim)) for _ in range(L)]
-    logits, hist, _ = synth.ngram_inputs(w.batch, synth.VOCAB, synth.NGRAM_SIZE, synth.NGRAM_WINDOW, 1)
-    lg, hi = logits.numpy(), hist.numpy()
-    steps = 0
-    t0 = time.perf_counter()
-    while True:
-        for l in range(L):
-            model.step(l, qkv[l][0], qkv[l][1], qkv[l][2], w.scale)
-        oracle.ngram_ban(lg, hi, None, synth.NGRAM_SIZE, synth.NGRAM_WINDOW)
-        steps += 1
-        el = time.perf_counter() - t0
-        if (el >= seconds and steps >= 2) or (max_steps and steps >= max_steps):
-            break
-    rate = steps / el * (L / w.layers)  # full-model decode steps per second
-    return rate, steps, el, oracle.num_threads(), L
+    nproc, model = host_cpu()
+    return {"value": sample.rate(), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "nproc": nproc, "cpu_model": model, "sample": sample.describe()}
 
 
 # --------------------------------------------------------------------------
@@ -454,13 +530,18 @@ def run_ours(args, rank, world, local_rank):
     s = torch.cuda.Stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    # ---- prefill (fills the caches of the main workload), then decode from t = 0
+    # ---- prefill (fills the caches of the main workload), then the ring's
+    # warm-up: W tokens appended after the prompt (untimed), so that every
+    # timed token overwrites the oldest ring entry and attends over exactly
+    # P_b + W keys (steady state)
     rig = DecodeRig(w, 0, "prefill", s)
     pf_ms = rig.prefill_all(flush)
     rig.capture()
+    fill_ring(rig)
     sampler = ClockSampler(dev if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dev]))
     ms, ts, clocks = timed_tokens(rig, args.steps, args.warmup, flush, sampler)
+    decode_from_t = min(ts[0])
     total_ms = max_over_ranks(sum(ms))
     value = aggregate_rate(args.steps, total_ms, world)
     kv_bytes = sum(w.layers * kv_bytes_per_layer(w, t) for t in ts)
@@ -492,7 +573,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": w.name, "batch": w.batch, "layers": w.layers, "heads": w.heads,
                    "head_dim": w.head_dim, "prefill_len": list(w.prefill_lens)[:4],
                    "window": w.window, "decode_steps_timed": args.steps,
-                   "decode_from_t": 0, "step": "one token: all layers' rswa_decode_step + "
+                   "decode_from_t": decode_from_t, "steady_state": decode_from_t >= w.window,
+                   "step": "one token: all layers' rswa_decode_step + "
                    "rswa_advance + rswa_ngram_mask (n=35, window=128) as one CUDA graph",
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
                    "parallelism": f"replicas x{world}",
@@ -521,6 +603,8 @@ def run_ours(args, rank, world, local_rank):
     also = []
     if world == 1 and args.also != "none":
         for name in args.also.split(","):
+            if name == w.name:
+                continue  # the headline already measured it
             if name == "continuous_batching":
                 also.append(run_continuous_batching(args, s, hbm_peak))
             elif name == "ngram_topk":
@@ -538,10 +622,9 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- CPU oracle on this host (rank 0, N = 1)
     if world == 1 and rank == 0 and args.cpu_seconds > 0:
-        rate, n, el, cores, lps = cpu_oracle_rate(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"{n} decode steps x {lps} layers of {w.name} from t=0 "
-                                          f"(plus the n-gram ban) in {el:.1f} s"}
+        sample = OracleSample(w, 1, range(w.batch))
+        sample.run(seconds=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline_block(sample)
     return line
 
 
@@ -890,28 +973,39 @@ def run_also(w, args, flush, s, hbm_peak, tc_peak):
     return res
 
 
+def reference_sample(w: synth.Workload, steps_total: int, budget_s: float,
+                     mem_cap: float = 4e9) -> OracleSample:
+    """The largest sample of (layer, sequence) units whose `steps_total` steps
+    fit in `budget_s` seconds and whose FP64 caches fit in `mem_cap` bytes:
+    one unit is timed first, then the sample is built once."""
+    probe = OracleSample(w, 1, [int(max(range(w.batch), key=lambda b: w.prefill_lens[b]))])
+    probe.run(max_steps=1)
+    unit_s = probe.attn_s + probe.ban_s
+    del probe
+    by_time = int(budget_s / max(unit_s * steps_total, 1e-9))
+    by_mem = int(mem_cap // (16 * (max(w.prefill_lens) + w.window) * w.heads * w.head_dim))
+    units = max(1, min(by_time, by_mem, w.layers * w.batch))
+    seqs = min(w.batch, units)
+    layers = max(1, min(w.layers, units // seqs))
+    return OracleSample(w, layers, range(seqs))
+
+
 def run_reference(args):
     w = _workload(args)
-    # size the sample: measure one step, then choose layers per step so that
-    # warmup + steps fit in the time budget
-    rate1, _, el1, _, _ = cpu_oracle_rate(w, 0.0, max_steps=1, layers_per_step=1)
-    per_layer = el1
-    budget = args.reference_budget
-    total_steps = args.steps + args.warmup
-    lps = max(1, min(w.layers, int(budget / max(per_layer * total_steps, 1e-9))))
+    sample = reference_sample(w, args.steps + args.warmup, args.reference_budget)
     if args.warmup:
-        cpu_oracle_rate(w, 0.0, max_steps=args.warmup, layers_per_step=lps)
-    rate, n, el, cores, lps = cpu_oracle_rate(w, 0.0, max_steps=args.steps, layers_per_step=lps)
+        sample.run(max_steps=args.warmup)
+    sample.reset_timers()
+    sample.run(max_steps=args.steps)
+    rate = sample.rate()
     return {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": 0,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / n * 1e3 * (w.layers / lps),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / rate,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "batch": w.batch, "layers": w.layers,
                                         "heads": w.heads, "head_dim": w.head_dim,
                                         "prefill_len": list(w.prefill_lens)[:4], "window": w.window},
-        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"each step: {lps} of {w.layers} layers of {w.name} "
-                                   f"(batch {w.batch}) + the n-gram ban; rate scaled to all layers"},
+        "cpu_baseline": cpu_baseline_block(sample),
         "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -919,13 +1013,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4096)
+    ap.add_argument("--steps", type=int, default=2048)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="single_page_decode")
+    ap.add_argument("--workload", default="near_max_context")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (small profiling runs)")
-    ap.add_argument("--also", default="multi_page_decode,near_max_context,ragged_serving,"
+    ap.add_argument("--also", default="single_page_decode,multi_page_decode,ragged_serving,"
                                       "continuous_batching,ngram_topk,rope,standard_swa,"
                                       "keysplit")
     ap.add_argument("--also-steps", type=int, default=40)
