@@ -145,9 +145,13 @@ cudaError_t launch_advance_rope(const DeviceView &v, cudaStream_t s);
 // (rotated keys, RoPE), which holds kc_rows rows of d elements.
 cudaError_t launch_prefill_simt(const DeviceView &v, const void *q, const void *k,
                                 const void *vv, void *out, const void *kc, cudaStream_t s);
+// The bf16 d = 128 prefill on the tensor cores.  It also fills cache slots
+// [0, P_b) of kc / vc (which hold kc_rows rows of d elements) with the
+// prompt's K / V; k_from_cache: K is read from kc (rotated keys, RoPE) and
+// only V is stored.
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, const int4 *blocks, int n_blocks, const void *kc,
-                              int64_t kc_rows, cudaStream_t s);
+                              void *out, const int4 *blocks, int n_blocks, void *kc, void *vc,
+                              int k_from_cache, int64_t kc_rows, cudaStream_t s);
 
 // Prefill work list of the tensor-core kernel: blocks of two consecutive
 // 128-row query tiles of one (b, h), in launch order.

@@ -36,6 +36,7 @@
 #include "internal.h"
 #include "ptx.cuh"
 #include "tcgen05.cuh"
+#include "tmap.h"
 
 namespace rswa {
 namespace {
@@ -83,7 +84,9 @@ struct PrefillTcArgs {
   DeviceView v;
   const int4 *blocks;  // (b, h, first query tile, number of tiles 1|2)
   __nv_bfloat16 *out;
+  __nv_bfloat16 *kc, *vc;  // this layer's caches (prompt rows of a ragged last tile)
   int k_from_cache;    // K tiles from the layer's cache (rotated keys) instead of k
+  int store_k, store_v;  // store the block's own K / V tiles into the cache
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *err,
@@ -119,7 +122,9 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const PrefillTcArgs a) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_kc,
+                      const __grid_constant__ CUtensorMap tm_vc, const PrefillTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // dynamic shared memory is only 16-byte aligned: round up to 1024 for the swizzle atoms
   PrefillSmem &sm = *reinterpret_cast<PrefillSmem *>(
@@ -139,6 +144,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int j0 = v.swa ? max(0, qt0 * kTile - v.W + 1) / kTile : 0;
   const int n_kv_a = qt0 + 1 - j0, n_kv_b = ntiles > 1 ? qt0 + 2 - j0 : 0;
   const int n_kv_all = qt0 + ntiles - j0;
+  // The cache fill (prompt K/V into cache slots [0, P_b)) rides on the loads:
+  // a block's last key tiles are its own query tiles qt0 .. qt0 + ntiles - 1
+  // (the diagonal), which no other block owns, so every prompt tile is stored
+  // exactly once.  They are the last loads of both rings, so their slots are
+  // never refilled.  A whole tile goes out by TMA store from the shared-memory
+  // tile the MMAs read; the rows of a ragged last tile (its rest would land
+  // in ring slots) by plain stores in the epilogue.
+  const int64_t crow0 = (int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W);
+  const int n_full_tiles = P / kTile;  // tiles lying wholly in the prompt
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
@@ -219,10 +233,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_addr0 = smem_u32(sm.q[0]);
+      // key tile j0 + it lands in K slot it mod 2 / V slot it mod 3; send it to
+      // the cache if it is one of this block's whole prompt tiles
+      bool stored = false;
+      auto store_tile = [&](const CUtensorMap *tm, const uint8_t *src, int it) {
+        const int kt = j0 + it;
+        if (kt < qt0 || kt >= n_full_tiles) return;
+        const int y = (int)(crow0 + (int64_t)kt * kTile);
+        tc::tma_store_2d(tm, src, 0, y);
+        tc::tma_store_2d(tm, src + kHalfBytes, 64, y);
+        stored = true;
+      };
       bool ok = wait_bar(&sm.q_full, 0, v.err, dead) &&
                 wait_bar(&sm.k_full[0], 0, v.err, dead);
       if (ok) {
         tc::fence_after_sync();
+        if (a.store_k) store_tile(&tm_kc, sm.k[0], 0);
         for (int x = 0; x < ntiles; ++x) {
           issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[0]));
           tc::commit(&sm.s_full[x]);
@@ -234,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s1 = (j + 1) % kKStages;   // K stage of tile j + 1
         bool k1_ready = false;  // K_{j+1} waited for
         if (!(ok = wait_bar(&sm.v_full[s], (j / kVStages) & 1, v.err, dead))) break;
+        if (a.store_v) store_tile(&tm_vc, sm.v[s], j);
         for (int x = 0; x < ntiles; ++x) {
           const int nkv = x == 0 ? n_kv_a : n_kv_b;
           if (j >= nkv) continue;
@@ -248,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(ok = wait_bar(&sm.k_full[s1], ((j + 1) / kKStages) & 1, v.err, dead))) break;
               tc::fence_after_sync();
               k1_ready = true;
+              if (a.store_k) store_tile(&tm_kc, sm.k[s1], j + 1);
             }
             issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[s1]));
             tc::commit(&sm.s_full[x]);
@@ -258,6 +286,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (k1_ready) tc::commit(&sm.k_empty[s1]);
       }
       tc::commit(&sm.mma_done);
+      if (stored) {
+        tc::store_commit();
+        tc::store_wait_read();  // the tiles stay in shared memory until read
+      }
       mbar_wait_bounded(&sm.mma_done, 0, v.err, RSWA_DEVERR_TIMEOUT);
     }
   } else {
@@ -391,6 +423,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // ragged last prompt tile (query tile qt of this warpgroup): rows
+    // [qt * 128, P) of its K / V into the cache, from its ring slots
+    const int rem = P - qt * kTile;
+    if (ok && x < ntiles && rem > 0 && rem < kTile && (a.store_k || a.store_v)) {
+      const int it = qt - j0;  // its load index in both rings
+      const int ks = it % kKStages, vs = it % kVStages;
+      const bool kr = !a.store_k || wait_bar(&sm.k_full[ks], (it / kKStages) & 1, v.err, dead);
+      const bool vr = !a.store_v || wait_bar(&sm.v_full[vs], (it / kVStages) & 1, v.err, dead);
+      if (kr && vr && r < rem) {
+        const int64_t grow = crow0 + (int64_t)qt * kTile + r;
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t off = (uint32_t)(c >> 3) * kHalfBytes + (uint32_t)r * 128u +
+                               ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+          if (a.store_k)
+            *reinterpret_cast<uint4 *>(a.kc + grow * kD + 8 * c) =
+                *reinterpret_cast<const uint4 *>(sm.k[ks] + off);
+          if (a.store_v)
+            *reinterpret_cast<uint4 *>(a.vc + grow * kD + 8 * c) =
+                *reinterpret_cast<const uint4 *>(sm.v[vs] + off);
+        }
+      }
+    }
   }
 
   tc::fence_before_sync();
@@ -399,50 +454,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tc::tmem_dealloc(tbase, kTmemCols);
 }
 
-// ------------------------------------------------------------ host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
-
 // [tokens][H * 128] bf16 activations, 64 x 128 boxes, 128-byte swizzle.
 bool make_tmap(CUtensorMap *m, const void *base, int64_t tokens, int H) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)H * kD, (cuuint64_t)tokens};
-  const cuuint64_t strides[1] = {(cuuint64_t)H * kD * 2};
-  const cuuint32_t box[2] = {64, kTile};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tmap_bf16(m, base, tokens, H, kTile);
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k, const void *vv,
-                              void *out, const int4 *blocks, int n_blocks, const void *kc,
-                              int64_t kc_rows, cudaStream_t s) {
+                              void *out, const int4 *blocks, int n_blocks, void *kc, void *vc,
+                              int k_from_cache, int64_t kc_rows, cudaStream_t s) {
   if (n_blocks == 0) return cudaSuccess;
   if (v.D != kD || v.dtype != RSWA_BF16) return cudaErrorInvalidValue;
-  if (kc && (kc_rows < 1 || kc_rows >= (int64_t(1) << 31))) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
-  // the cache as [kc_rows][1 x 128]: the same encoding with H = 1
-  const bool k_ok = kc ? make_tmap(&tk, kc, kc_rows, 1) : make_tmap(&tk, k, v.total_tokens, v.H);
-  if (!make_tmap(&tq, q, v.total_tokens, v.H) || !k_ok || !make_tmap(&tv, vv, v.total_tokens, v.H))
+  if (!kc || !vc || kc_rows < 1 || kc_rows >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv, tkc, tvc;
+  // the caches as [kc_rows][1 x 128]: the same encoding with H = 1
+  const bool k_ok = k_from_cache ? make_tmap(&tk, kc, kc_rows, 1)
+                                 : make_tmap(&tk, k, v.total_tokens, v.H);
+  if (!make_tmap(&tq, q, v.total_tokens, v.H) || !k_ok ||
+      !make_tmap(&tv, vv, v.total_tokens, v.H) || !make_tmap(&tkc, kc, kc_rows, 1) ||
+      !make_tmap(&tvc, vc, kc_rows, 1))
     return cudaErrorInvalidValue;
   const int smem = (int)sizeof(PrefillSmem) + 1024;
   // the attribute holds per device for the life of the process: set it once
@@ -455,8 +486,10 @@ cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k,
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  PrefillTcArgs args{v, blocks, (__nv_bfloat16 *)out, kc ? 1 : 0};
-  prefill_tc_kernel<<<n_blocks, kThreads, smem, s>>>(tq, tk, tv, args);
+  // RoPE: the rotated keys are in the cache already; only V is stored
+  PrefillTcArgs args{v,  blocks, (__nv_bfloat16 *)out, (__nv_bfloat16 *)kc, (__nv_bfloat16 *)vc,
+                     k_from_cache, k_from_cache ? 0 : 1, 1};
+  prefill_tc_kernel<<<n_blocks, kThreads, smem, s>>>(tq, tk, tv, tkc, tvc, args);
   return cudaGetLastError();
 }
 

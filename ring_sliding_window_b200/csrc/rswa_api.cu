@@ -436,7 +436,12 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
   if (current_device() != s->device) return RSWA_EINVAL;
   cudaStream_t st = (cudaStream_t)stream;
   void *kc = s->k_cache[(size_t)layer];
-  cudaError_t e = launch_cache_fill(s->dv, k, v, kc, s->v_cache[(size_t)layer], st);
+  void *vc = s->v_cache[(size_t)layer];
+  const int64_t kc_rows = (int64_t)s->cfg.num_heads * s->pool_slots;
+  // the tensor-core kernel stores the prompt K/V into the cache itself; the
+  // CUDA-core kernel takes a separate cache-fill pass
+  const bool fused_fill = s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128;
+  cudaError_t e = fused_fill ? cudaSuccess : launch_cache_fill(s->dv, k, v, kc, vc, st);
   // RoPE: rotated k overwrites the cache's prompt slots, rotated q goes to
   // `out`; attention then reads q from `out` and k from the cache
   const bool rope = s->dv.rope != RSWA_ROPE_NONE;
@@ -444,9 +449,9 @@ rswa_status rswa_prefill(rswa_state *s, int32_t layer, const void *q, const void
   const void *qa = rope ? (const void *)out : q;
   const void *kca = rope ? (const void *)kc : nullptr;
   if (e == cudaSuccess) {
-    if (s->cfg.dtype == RSWA_BF16 && s->cfg.head_dim == 128)
-      e = launch_prefill_tc(s->dv, qa, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, kca,
-                            (int64_t)s->cfg.num_heads * s->pool_slots, st);
+    if (fused_fill)
+      e = launch_prefill_tc(s->dv, qa, k, v, out, s->dv.pf_blocks, s->dv.n_pf_blocks, kc, vc,
+                            rope ? 1 : 0, kc_rows, st);
     else
       e = launch_prefill_simt(s->dv, qa, k, v, out, kca, st);
   }
