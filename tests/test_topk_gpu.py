@@ -113,6 +113,21 @@ def test_topk_vocab_sizes_and_clusters(vocab):
         assert err.item() == 0
 
 
+@pytest.mark.parametrize("rows,vocab", [(300, 16), (513, 1000), (64, 4100)])
+def test_topk_many_short_rows_per_cta(rows, vocab):
+    """Many short rows (one to two CTAs each) and a row of 4,100 columns over
+    one cluster of CTAs; a repeat planted in every history, k and
+    mask_in_place over their range."""
+    g = torch.Generator().manual_seed(rows * 7 + vocab)
+    logits = torch.randn(rows, vocab, generator=g)
+    window, n = 12, 3
+    hist = torch.randint(0, vocab, (rows, window), generator=g, dtype=torch.int32)
+    hist[:, 3:5] = hist[:, window - 2:]  # the last 2 tokens also at 3..4: bans hist[5]
+    for k in sorted({1, 5, min(64, vocab)}):
+        for mask_in_place in (False, True):
+            _check(logits, hist, None, n, window, k, mask_in_place)
+
+
 def test_topk_ties_nan_inf_and_ragged_histories():
     vocab, rows, n, window = 5000, 8, 3, 32
     g = torch.Generator().manual_seed(11)
