@@ -289,6 +289,11 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
   const int rank = (int)(blockIdx.x % (unsigned)C);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int col0 = rank * kChunk;
+  // programmatic dependent launch: the previous kernel (which may have written
+  // the logits or the history) has completed past this point, and the next
+  // launch may start scheduling its CTAs while this one runs
+  grid_dependency_wait();
+  allow_dependents();
   // arrive now, wait before the first remote store: no CTA then writes into a
   // peer that has not started, and the wait costs nothing by that time
   cluster_arrive_relaxed();
@@ -402,6 +407,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int tid = threadIdx.x;
   const int col0 = rank * kChunk;
   const float *lrow = a.logits + (int64_t)row * a.ld;
+  grid_dependency_wait();  // as in the greedy kernel
+  allow_dependents();
   cluster_arrive_relaxed();
   if (tid == 0) {
     n_cand = 0;
@@ -581,13 +588,15 @@ cudaError_t launch_ngram_topk(float *logits, int64_t ld, const int32_t *history,
     if (e != cudaSuccess) return e;
   }
   lc.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
-  lc.numAttrs = 1;
+  lc.numAttrs = 2;
   return cudaLaunchKernelEx(&lc, kernel, a);
 }
 
