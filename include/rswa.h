@@ -456,9 +456,15 @@ rswa_status rswa_decode_step_noalloc(const rswa_config *cfg, const int64_t *pref
  * issue none of their cache copies, so every bounded wait in them runs out
  * (about 1 s): the kernel records RSWA_DEVERR_TIMEOUT, finishes, and
  * rswa_check_device_error returns RSWA_ETIMEOUT; outputs of those steps are
- * garbage, the cache is untouched apart from the ring write.  flags = 0
- * restores normal operation.  Enqueued on `stream` (pageable copy). */
+ * garbage, the cache is untouched apart from the ring write.
+ * RSWA_FAULT_DROP_PREFILL_LOADS: subsequent tensor-core prefills (bf16,
+ * d = 128) of this state issue none of their tile loads: every bounded wait
+ * runs out, the kernel records RSWA_DEVERR_TIMEOUT, frees its tensor memory
+ * and returns; the outputs and the cache's prompt slots of those calls are not
+ * written.  flags = 0 restores normal operation.  Enqueued on `stream`
+ * (pageable copy). */
 #define RSWA_FAULT_DROP_DECODE_COPIES 1
+#define RSWA_FAULT_DROP_PREFILL_LOADS 2
 rswa_status rswa_debug_inject_fault(rswa_state *state, int32_t flags, void *stream);
 
 /* Bits of a device error word. */

@@ -189,11 +189,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // waits behind a V slot that is still in use (and the other way round).
     if (lane == 0) {
       const bool is_k = warp == kProducerWarp;
+      // test-only fault injection: no loads at all, so every wait on them
+      // runs out (bounded) and the kernel takes its timeout path
+      const bool drop_loads = (*v.fault & RSWA_FAULT_DROP_PREFILL_LOADS) != 0;
       const int xh = h * kD;
       const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
       const int nst = is_k ? kKStages : kVStages;
       tc::prefetch_tmap(tm);
-      if (is_k) {
+      if (is_k && !drop_loads) {
         tc::prefetch_tmap(&tm_q);
         mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(ntiles * kTileBytes));
         for (int x = 0; x < ntiles; ++x) {
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int x0 = from_cache ? 0 : xh;
       const int y0 = from_cache ? (int)((int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W))
                                 : tok0;
-      for (int j = 0; j < n_kv_all; ++j) {
+      for (int j = 0; !drop_loads && j < n_kv_all; ++j) {
         const int s = j % nst;
         uint64_t *empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
         uint64_t *full = is_k ? &sm.k_full[s] : &sm.v_full[s];
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = j + 1;
       }
       // every load issued has landed before the CTA may exit (bounded)
-      if (is_k) mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
+      if (is_k && !drop_loads) mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
       for (int s = 0; s < nst && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / nst) * nst;
         mbar_wait_bounded(is_k ? &sm.k_full[s] : &sm.v_full[s], (last / nst) & 1, v.err,

@@ -629,7 +629,8 @@ rswa_status rswa_check_device_error(rswa_state *s, void *stream) {
 }
 
 rswa_status rswa_debug_inject_fault(rswa_state *s, int32_t flags, void *stream) {
-  if (!s || (flags & ~RSWA_FAULT_DROP_DECODE_COPIES) != 0) return RSWA_EINVAL;
+  if (!s || (flags & ~(RSWA_FAULT_DROP_DECODE_COPIES | RSWA_FAULT_DROP_PREFILL_LOADS)) != 0)
+    return RSWA_EINVAL;
   if (current_device() != s->device) return RSWA_EINVAL;
   // the host value is staged by the copy before the call returns
   return from_cuda(cudaMemcpyAsync((int *)s->dv.fault, &flags, sizeof(int32_t),

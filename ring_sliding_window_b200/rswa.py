@@ -40,6 +40,7 @@ RSWA_ATTN_RING, RSWA_ATTN_STANDARD_SWA = 0, 1
 RSWA_ROPE_NONE, RSWA_ROPE_ABSOLUTE, RSWA_ROPE_SLOT = 0, 1, 2
 RSWA_TOPK_MAX, RSWA_TOPK_MAX_VOCAB = 64, 262144
 RSWA_FAULT_DROP_DECODE_COPIES = 1
+RSWA_FAULT_DROP_PREFILL_LOADS = 2
 RSWA_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
