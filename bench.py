@@ -438,32 +438,35 @@ def host_cpu():
 
 class OracleSample:
     """The oracle as it stands, on this host's cores, over a bounded sample of
-    a workload: `layers` layers of the sequences `seqs`, each with every head,
-    prefilled with N(0,1) keys and values, then decoded from t = 0.  A step
-    runs the sampled layers' ring steps and the n-gram ban of the whole batch
-    (n = 35, window = 128).  The attention part is scaled to the whole model by
-    its key count (sampled keys / all keys of all layers), the ban is counted
-    once per step, so `rate()` is full-model decode steps per second."""
+    a workload: `layers` layers of the sequences `seqs`, with `heads` of the
+    heads (all by default; heads are independent), prefilled with N(0,1) keys
+    and values, then decoded from t = 0.  A step runs the sampled layers' ring
+    steps and the n-gram ban of the whole batch (n = 35, window = 128).  The
+    attention part is scaled to the whole model by its key count (sampled keys
+    / all keys of all layers and heads), the ban is counted once per step, so
+    `rate()` is full-model decode steps per second."""
 
-    def __init__(self, w: synth.Workload, layers: int, seqs):
+    def __init__(self, w: synth.Workload, layers: int, seqs, heads: int = 0):
         import numpy as np
 
         import oracle
         self.w, self.layers, self.seqs = w, layers, list(seqs)
+        self.heads = heads if heads > 0 else w.heads
+        H = self.heads
         rng = np.random.default_rng(0)
         plens = [w.prefill_lens[b] for b in self.seqs]
-        self.model = oracle.RingModel(plens, w.window, layers, w.heads, w.head_dim)
+        self.model = oracle.RingModel(plens, w.window, layers, H, w.head_dim)
         for l in range(layers):
             for i, P in enumerate(plens):
-                self.model.prefill(l, i, rng.standard_normal((P, w.heads, w.head_dim)),
-                                   rng.standard_normal((P, w.heads, w.head_dim)))
+                self.model.prefill(l, i, rng.standard_normal((P, H, w.head_dim)),
+                                   rng.standard_normal((P, H, w.head_dim)))
         nb = len(plens)
-        self.qkv = [rng.standard_normal((3, nb, w.heads, w.head_dim)) for _ in range(layers)]
+        self.qkv = [rng.standard_normal((3, nb, H, w.head_dim)) for _ in range(layers)]
         logits, hist, _ = synth.ngram_inputs(w.batch, synth.VOCAB, synth.NGRAM_SIZE,
                                              synth.NGRAM_WINDOW, 1)
         self.lg, self.hi = logits.numpy(), hist.numpy()
         keys = lambda ps: sum(P + w.window for P in ps)  # noqa: E731 (steady-state keys)
-        self.fraction = layers * keys(plens) / (w.layers * keys(w.prefill_lens))
+        self.fraction = layers * H * keys(plens) / (w.layers * w.heads * keys(w.prefill_lens))
         self.steps, self.attn_s, self.ban_s = 0, 0.0, 0.0
 
     def run(self, seconds: float = 0.0, max_steps=None):
@@ -498,8 +501,9 @@ class OracleSample:
 
     def describe(self) -> str:
         w = self.w
+        heads = f"all {w.heads}" if self.heads == w.heads else f"{self.heads} of {w.heads}"
         return (f"{self.steps} decode steps of {self.layers} of {w.layers} layers x "
-                f"{len(self.seqs)} of {w.batch} sequences (all {w.heads} heads) of {w.name} "
+                f"{len(self.seqs)} of {w.batch} sequences ({heads} heads) of {w.name} "
                 f"from t = 0, plus the n-gram ban of the batch; {self.attn_s + self.ban_s:.1f} s. "
                 f"Attention scaled to the whole model by its key count "
                 f"(sample = {self.fraction:.4f} of the keys); the first W steps attend over "
@@ -977,14 +981,21 @@ def reference_sample(w: synth.Workload, steps_total: int, budget_s: float,
                      mem_cap: float = 4e9) -> OracleSample:
     """The largest sample of (layer, sequence) units whose `steps_total` steps
     fit in `budget_s` seconds and whose FP64 caches fit in `mem_cap` bytes:
-    one unit is timed first, then the sample is built once."""
-    probe = OracleSample(w, 1, [int(max(range(w.batch), key=lambda b: w.prefill_lens[b]))])
+    one unit is timed first, then the sample is built once.  When even one
+    unit is too slow, the sample keeps only some of its heads."""
+    longest = int(max(range(w.batch), key=lambda b: w.prefill_lens[b]))
+    probe = OracleSample(w, 1, [longest])
     probe.run(max_steps=1)
-    unit_s = probe.attn_s + probe.ban_s
+    unit_attn, unit_ban = probe.attn_s, probe.ban_s
     del probe
-    by_time = int(budget_s / max(unit_s * steps_total, 1e-9))
+    by_time = int(budget_s / max((unit_attn + unit_ban) * steps_total, 1e-9))
     by_mem = int(mem_cap // (16 * (max(w.prefill_lens) + w.window) * w.heads * w.head_dim))
-    units = max(1, min(by_time, by_mem, w.layers * w.batch))
+    units = min(by_time, by_mem, w.layers * w.batch)
+    if units < 1:
+        # one layer of one sequence, as many heads as the budget allows
+        per_head = unit_attn / w.heads
+        heads = int((budget_s / steps_total - unit_ban) / max(per_head, 1e-9))
+        return OracleSample(w, 1, [longest], heads=max(1, min(w.heads, heads)))
     seqs = min(w.batch, units)
     layers = max(1, min(w.layers, units // seqs))
     return OracleSample(w, layers, range(seqs))
