@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace rswa {
 namespace {
@@ -25,6 +26,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                       int n, int window, int *err) {
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  // programmatic dependent launch: the previous kernel (which may have written
+  // the logits or the history) has completed past this point; the next launch
+  // may start scheduling meanwhile
+  grid_dependency_wait();
+  allow_dependents();
   if (row >= rows) return;
   const int32_t *hist = history + (int64_t)row * hist_ld;
   const int h = hist_len ? __ldg(hist_len + row) : window;
@@ -64,9 +70,17 @@ cudaError_t launch_ngram(float *logits, int64_t ld, const int32_t *history, int6
                          int *err, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
   const int blocks = (rows + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  ngram_mask_kernel<<<blocks, kWarpsPerBlock * 32, 0, s>>>(logits, ld, history, hist_ld, hist_len,
-                                                          rows, vocab, n, window, err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)blocks);
+  lc.blockDim = dim3(kWarpsPerBlock * 32);
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, ngram_mask_kernel, logits, ld, history, hist_ld, hist_len, rows,
+                            vocab, n, window, err);
 }
 
 }  // namespace rswa
