@@ -81,3 +81,38 @@ def test_prefill_full_size_sampled_rows(name):
                 assert err <= tol_for(w1.dtype), (b, h, i, err)
         kc = st.cache_view(0, "k", b, 0)
         assert torch.equal(kc[:P], k[sl[b], 0])
+
+
+@pytest.mark.slow
+def test_prefill_ragged_long_prompts_cache_fill_and_sampled_rows():
+    """Long ragged prompts as in the ragged-serving mix (lengths drawn from
+    [1,024, 16,384], none a multiple of 128), 10 heads x 128, bf16: enough
+    blocks for the tensor-core kernel's tile pairs.  The cache's prompt slots
+    [0, P_b) of every (b, h) ring hold the prompt's K and V bit for bit (the
+    fill is fused into the prefill: whole tiles by TMA store, the ragged last
+    tile row by row), and sampled rows match the oracle."""
+    from ring_sliding_window_b200 import rswa
+    lens = (1031, 16383, 4097, 9001, 2053, 12289)
+    w = synth.Workload("ragged_long", 27, torch.bfloat16, len(lens), 1, 10, 128, 128, lens, 0)
+    st = _state(w)
+    q, k, v = synth.prefill_qkv(w, 0, "cuda")
+    out = torch.empty_like(q)
+    st.prefill(0, q, k, v, out)
+    torch.cuda.synchronize()
+    assert st.check() == 0
+    sl = seq_slices(lens)
+    for b, P in enumerate(lens):
+        for h in range(w.heads):
+            assert torch.equal(st.cache_view(0, "k", b, h)[:P], k[sl[b], h]), (b, h)
+            assert torch.equal(st.cache_view(0, "v", b, h)[:P], v[sl[b], h]), (b, h)
+    rng = np.random.default_rng(11)
+    for b in (0, 1, 3):
+        P = lens[b]
+        h = int(rng.integers(0, w.heads))
+        kk, vv = f64(k[sl[b], h]), f64(v[sl[b], h])
+        rows = sorted({0, P - 1, (P // 128) * 128, (P // 128) * 128 - 1, int(rng.integers(0, P))})
+        for i in rows:
+            ref = oracle.attend(f64(q[sl[b].start + i, h]), kk[:i + 1], vv[:i + 1], w.scale)
+            err = np.max(np.abs(f64(out[sl[b].start + i, h]) - ref))
+            assert err <= tol_for(w.dtype), (b, h, i, err)
+    st.close()
