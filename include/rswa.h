@@ -415,7 +415,10 @@ const char *rswa_last_cuda_error(void);
  * synchronise the device.
  *
  * Same computation as rswa_decode_step for ONE layer, without a state: the
- * caller passes the ring position explicitly and advances it itself.
+ * caller passes the ring position explicitly and advances it itself.  It is
+ * always the ring attention of the method, with keys and queries used as
+ * given: the RoPE and attention-mode settings of rswa_state_set_rope and
+ * rswa_state_set_attention belong to a state and do not apply here.
  *  cfg           : as for rswa_state_create (num_layers is ignored).
  *  prefill_len   : host [B], P_b.
  *  n_generated   : host [B], t_b = tokens generated before this step; the

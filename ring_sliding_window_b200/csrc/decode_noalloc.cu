@@ -51,6 +51,19 @@ rswa_status scratch_for_device(int dev, uint8_t **out) {
   return RSWA_OK;
 }
 
+// Resident decode CTAs per SM for (device, dtype, head_dim), worked out once:
+// the query sets a function attribute and runs an occupancy calculation,
+// which a latency-bound serving loop should not repeat at every step.
+int g_ctas_per_sm[kMaxDevices][4] = {};
+
+int ctas_per_sm_cached(int dev, int dtype, int head_dim) {
+  const int key = (dtype == RSWA_BF16 ? 0 : 2) + (head_dim == 128 ? 0 : 1);
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  int &n = g_ctas_per_sm[dev][key];
+  if (n == 0) n = decode_ctas_per_sm(dtype, head_dim);
+  return n;
+}
+
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -117,9 +130,10 @@ extern "C" rswa_status rswa_decode_step_noalloc(const rswa_config *cfg,
     if (n_generated[b] < 0) return RSWA_EINVAL;
   const int dev = current_device();
   if (dev < 0) return RSWA_ECUDA;
+  if (dev >= kMaxDevices) return RSWA_EINVAL;
 
-  const DecodePlan plan =
-      plan_decode(cfg, prefill_len, nullptr, sm_count(dev), decode_ctas_per_sm(cfg->dtype, cfg->head_dim));
+  const DecodePlan plan = plan_decode(cfg, prefill_len, nullptr, sm_count(dev),
+                                      ctas_per_sm_cached(dev, cfg->dtype, cfg->head_dim));
   const NoAllocLayout ws = noalloc_layout(cfg, plan);
   if (ws.total > kNoAllocScratchBytes) return RSWA_ENOMEM;  // batch too large for the array
 
