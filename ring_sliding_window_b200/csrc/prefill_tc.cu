@@ -48,7 +48,14 @@ constexpr int kVStages = 3;  // V ring depth: a V tile is held until PV_B is don
                              // 32 KB tile load takes ~2.8 us under full load
 constexpr int kHalfBytes = kTile * 64 * 2;   // one 64-column swizzled half: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;   // 32 KB
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;       // three warpgroups: softmax A, softmax B, the rest
+constexpr int kLaunchRegs = 168;    // registers per thread at launch (65,536 / 384, rounded down to 8)
+// Registers per thread after the split: the softmax warpgroups hold a whole
+// 128-score row in registers; the loader / MMA warpgroup needs few.
+constexpr int kSoftmaxRegs = 224;
+constexpr int kAuxRegs = 56;
+static_assert(256 * kSoftmaxRegs + 128 * kAuxRegs <= kThreads * kLaunchRegs,
+              "register split above the launch's registers");
 constexpr int kProducerWarp = 8;   // Q and K loads
 constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10; // V loads
@@ -183,6 +190,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = sm.tmem_base;
   volatile int *dead = &sm.dead;
 
+  // Registers move from the loader / MMA warpgroup (warps 8-11; warp 11 has
+  // no role) to the two softmax warpgroups.  Each warpgroup changes its count
+  // at the top of its own branch, so the compiler allocates each branch
+  // within its own count.
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kAuxRegs));
   if (warp == kProducerWarp || warp == kVProducerWarp) {
     // ------------------------------------------------------------ producers
     // warp 8 loads Q and the K ring, warp 10 the V ring, so a K load never
@@ -295,7 +308,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mbar_wait_bounded(&sm.mma_done, 0, v.err, RSWA_DEVERR_TIMEOUT);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ------------------------------------------------------------ softmax
     const int x = warp >> 2;          // query tile of this warpgroup (0 = A, 1 = B)
     const int wq = warp & 3;          // warp inside the warpgroup = TMEM lane quarter
@@ -487,6 +502,12 @@ cudaError_t launch_prefill_tc(const DeviceView &v, const void *q, const void *k,
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // the register split inside the kernel assumes kLaunchRegs per thread at
+    // launch; with fewer, its setmaxnreg.inc could never be satisfied
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, prefill_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kLaunchRegs) return cudaErrorInvalidConfiguration;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   // RoPE: the rotated keys are in the cache already; only V is stored
