@@ -34,8 +34,9 @@ __device__ __forceinline__ float2 rope_cs(int64_t pos, int i, int d, float theta
 // Thread i < d/2 reduces the run's first angle for pair i once (double
 // sincos) and walks the run with the angle-addition recurrence in double
 // precision (kRun steps add a few 1e-16), leaving float (cos, sin) in shared
-// memory; then all threads rotate q and k of every head of the run, with
-// consecutive threads on consecutive elements.
+// memory; then all threads rotate q and k of every head of the run, each
+// thread 16 bytes of both halves of a row at a time, consecutive threads on
+// consecutive 16-byte pieces.
 constexpr int kRun = 64;
 
 template <typename T>
@@ -68,22 +69,36 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncthreads();
-  const int per_pos = v.H * half;
+  // one item = 16 bytes of a half row (8 bf16 or 4 fp32 pairs) of one head
+  constexpr int VW = Chunk<T>::N;
+  const int cph = half / VW;  // items per half row
+  const int per_pos = v.H * cph;
   const int64_t tok0 = v.tok_base[b] + p0;
   const int64_t krow0 = (int64_t)v.H * v.slot_base[b] + p0;
   for (int e = threadIdx.x; e < n * per_pos; e += blockDim.x) {
     const int j = e / per_pos;
     const int rem = e - j * per_pos;
-    const int h = rem / half, ii = rem - h * half;
-    const float2 r = cs[j][ii];
+    const int h = rem / cph, ii = (rem - h * cph) * VW;
     const int64_t src = ((tok0 + j) * v.H + h) * v.D + ii;
     const int64_t dst = (krow0 + (int64_t)h * (P + v.W) + j) * v.D + ii;
-    const float qa = to_float(q[src]), qb = to_float(q[src + half]);
-    const float ka = to_float(k[src]), kb = to_float(k[src + half]);
-    qr[src] = from_float<T>(qa * r.x - qb * r.y);
-    qr[src + half] = from_float<T>(qb * r.x + qa * r.y);
-    kc[dst] = from_float<T>(ka * r.x - kb * r.y);
-    kc[dst + half] = from_float<T>(kb * r.x + ka * r.y);
+    float qa[VW], qb[VW], ka[VW], kb[VW];
+    Chunk<T>::widen(*reinterpret_cast<const uint4 *>(q + src), qa);
+    Chunk<T>::widen(*reinterpret_cast<const uint4 *>(q + src + half), qb);
+    Chunk<T>::widen(*reinterpret_cast<const uint4 *>(k + src), ka);
+    Chunk<T>::widen(*reinterpret_cast<const uint4 *>(k + src + half), kb);
+    float q1[VW], q2[VW], k1[VW], k2[VW];
+#pragma unroll
+    for (int t = 0; t < VW; ++t) {
+      const float2 r = cs[j][ii + t];
+      q1[t] = qa[t] * r.x - qb[t] * r.y;
+      q2[t] = qb[t] * r.x + qa[t] * r.y;
+      k1[t] = ka[t] * r.x - kb[t] * r.y;
+      k2[t] = kb[t] * r.x + ka[t] * r.y;
+    }
+    *reinterpret_cast<uint4 *>(qr + src) = Chunk<T>::narrow(q1);
+    *reinterpret_cast<uint4 *>(qr + src + half) = Chunk<T>::narrow(q2);
+    *reinterpret_cast<uint4 *>(kc + dst) = Chunk<T>::narrow(k1);
+    *reinterpret_cast<uint4 *>(kc + dst + half) = Chunk<T>::narrow(k2);
   }
 }
 
