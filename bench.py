@@ -511,6 +511,42 @@ class OracleSample:
                 f"{min(w.prefill_lens) + w.window} at most)")
 
 
+def oracle_prefill_sample(w: synth.Workload, seconds: float) -> dict:
+    """The oracle's causal prefill on this host's cores, over a bounded sample
+    of the workload's prefill: blocks of 64 consecutive query rows of one head
+    of the first sequence, at evenly spaced positions of its prompt (N(0,1)
+    q, k, v), run until `seconds` have passed.  A row i costs 4*d*(i + 1)
+    FLOPs (causal keys only, as the GPU figure counts them), so the rate is
+    FLOP/s of the same work and the full prefill time is extrapolated from
+    it."""
+    import numpy as np
+
+    import oracle
+    P, d = w.prefill_lens[0], w.head_dim
+    rng = np.random.default_rng(1)
+    q, k, v = (rng.standard_normal((P, 1, d)) for _ in range(3))
+    block = min(64, P)
+    starts = [min(P - block, (P * j) // 8) for j in range(8)]
+    flops, rows, spent, j = 0, 0, 0.0, 0
+    while spent < seconds or j < len(starts):
+        lo = starts[j % len(starts)]
+        t0 = time.perf_counter()
+        oracle.prefill(q, k, v, w.scale, lo, lo + block)
+        spent += time.perf_counter() - t0
+        flops += sum(4 * d * (i + 1) for i in range(lo, lo + block))
+        rows += block
+        j += 1
+    rate = flops / spent
+    nproc, model = host_cpu()
+    full = prefill_flops_per_layer(w) * w.layers
+    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "nproc": nproc, "cpu_model": model,
+            "sample": f"{rows} query rows of 1 of {w.heads} heads of sequence 0 "
+                      f"(P = {P}) in blocks of {block} at 8 evenly spaced positions; "
+                      f"{spent:.1f} s",
+            "extrapolated_full_prefill_s": full / rate}
+
+
 def cpu_baseline_block(sample: OracleSample) -> dict:
     import oracle
     nproc, model = host_cpu()
@@ -629,6 +665,7 @@ def run_ours(args, rank, world, local_rank):
         sample = OracleSample(w, 1, range(w.batch))
         sample.run(seconds=args.cpu_seconds)
         line["cpu_baseline"] = cpu_baseline_block(sample)
+        line["prefill"]["cpu_baseline"] = oracle_prefill_sample(w, args.cpu_seconds / 2)
     return line
 
 
