@@ -277,6 +277,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool k1_ready = false;  // K_{j+1} waited for
         if (!(ok = wait_bar(&sm.v_full[s], (j / kVStages) & 1, v.err, dead))) break;
         if (a.store_v) store_tile(&tm_vc, sm.v[s], j);
+        // K_{j+1} has usually landed by now: taking it here keeps the barrier
+        // check out of the gap between P V and the next Q K^T of tile A (a
+        // wait issued right after a burst of MMAs costs 50-200 cycles).  If
+        // it has not, it is waited for there, as before.
+        if (j + 1 < n_kv_all && mbar_try_wait(&sm.k_full[s1], ((j + 1) / kKStages) & 1)) {
+          tc::fence_after_sync();
+          k1_ready = true;
+          if (a.store_k) store_tile(&tm_kc, sm.k[s1], j + 1);
+        }
         for (int x = 0; x < ntiles; ++x) {
           const int nkv = x == 0 ? n_kv_a : n_kv_b;
           if (j >= nkv) continue;
