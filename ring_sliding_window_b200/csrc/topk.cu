@@ -330,23 +330,56 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
 
 // Threshold T with exactly k of the n keys (which may repeat) at or above it
 // when the k-th largest key is unique among them, and at least k otherwise:
-// a radix select, 8 bits per pass from the top, stopping when the chosen
-// digit's bin holds exactly the keys still needed.  CTA-wide; keys in shared
-// memory; ends with a barrier.
+// a radix select over d = key - (smallest key), from the top bit of the
+// largest d down, 8 bits per pass, stopping when the chosen digit's bin holds
+// exactly the keys still needed.  Taking digits of d rather than of the key
+// spreads keys that share their leading bits (thread maxima of N(0, 1)
+// logits mostly share sign and exponent) over the bins from the first pass,
+// so the histogram atomics rarely collide.  CTA-wide; keys in shared memory;
+// ends with a barrier.
 __device__ unsigned long long cta_kth_threshold(const unsigned long long *keys, int n, int k,
-                                                uint32_t *hist, uint32_t *scan, uint32_t *sel) {
+                                                uint32_t *hist, uint32_t *scan, uint32_t *sel,
+                                                unsigned long long *span) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned long long lo = ~0ull, hi = 0;
+  for (int i = tid; i < n; i += kThreads) {
+    lo = min(lo, keys[i]);
+    hi = max(hi, keys[i]);
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  if (lane == 0) {  // span: 2 x kWarps
+    span[warp] = lo;
+    span[kWarps + warp] = hi;
+  }
+  __syncthreads();
+  lo = span[0];
+  hi = span[kWarps];
+  for (int i = 1; i < kWarps; ++i) {
+    lo = min(lo, span[i]);
+    hi = max(hi, span[kWarps + i]);
+  }
+  if (lo == hi) {
+    __syncthreads();  // span is rewritten by the next call
+    return lo;
+  }
+  // bits [lo_shift, hi_shift) of d form this pass's digit; the bits above
+  // are `prefix` for every key still in the running
+  int hi_shift = 64 - __clzll((long long)(hi - lo));
+  int lo_shift = hi_shift > 8 ? hi_shift - 8 : 0;
   unsigned long long prefix = 0;
   uint32_t need = (uint32_t)k;
-  int pass = 0;
-  for (;; ++pass) {
-    const int shift = 56 - 8 * pass;
+  for (;;) {
     hist[tid] = 0;
     __syncthreads();
+    const uint32_t mask = (1u << (hi_shift - lo_shift)) - 1u;
     for (int i = tid; i < n; i += kThreads) {
-      const unsigned long long key = keys[i];
-      if (pass == 0 || (key >> (shift + 8)) == prefix)
-        atomicAdd(&hist[(uint32_t)(key >> shift) & 0xFFu], 1u);
+      const unsigned long long d = keys[i] - lo;
+      if (hi_shift >= 64 || (d >> hi_shift) == prefix)
+        atomicAdd(&hist[(uint32_t)(d >> lo_shift) & mask], 1u);
     }
     __syncthreads();
     // bin (255 - tid); suffix sums = prefix scan of the reversed bins
@@ -369,13 +402,15 @@ __device__ unsigned long long cta_kth_threshold(const unsigned long long *keys, 
       sel[2] = cnt == need - (incl - cnt);
     }
     __syncthreads();
-    prefix = (prefix << 8) | sel[0];
+    prefix = (prefix << (hi_shift - lo_shift)) | sel[0];
     need = sel[1];
-    const bool done = sel[2] || pass == 7;
+    const bool done = sel[2] || lo_shift == 0;
+    hi_shift = lo_shift;
+    lo_shift = lo_shift > 8 ? lo_shift - 8 : 0;
     __syncthreads();  // sel and hist are rewritten by the next pass
     if (done) break;
   }
-  return prefix << (56 - 8 * pass);
+  return lo + (prefix << hi_shift);
 }
 
 // k > 1, one cluster per row:
@@ -393,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan[kWarps];
   __shared__ uint32_t sel[3];
+  __shared__ unsigned long long span[2 * kWarps];
   __shared__ unsigned long long thr;               // T, written by the leader into every CTA
   __shared__ uint32_t n_cand, n_top;               // leader: candidates received, selected
   __shared__ unsigned long long sorted[kTopkMax];
@@ -430,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   cluster_arrive_release();
   cluster_wait_acquire();
   if (rank == 0) {
-    const unsigned long long T = cta_kth_threshold(keybuf, C * kThreads, a.k, hist, scan, sel);
+    const unsigned long long T = cta_kth_threshold(keybuf, C * kThreads, a.k, hist, scan, sel, span);
     if (tid < C) st_cluster_u64(map_to_rank(&thr, tid), T);
   }
   cluster_arrive_release();
@@ -495,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     __syncthreads();
   } else {
-    const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel);
+    const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel, span);
     for (int i = tid; i < nc; i += kThreads) {
       const unsigned long long kk = keybuf[i];
       if (kk >= T2) {
@@ -522,22 +558,38 @@ __global__ void __launch_bounds__(kThreads, 4)
     prob[tid] = (val == -INFINITY || x0 == -INFINITY) ? 0.f : exp2f((val - x0) * a.inv_temp_log2e);
   }
   __syncthreads();
-  if (tid == 0 && a.token) {
-    int pick = 0;
-    if (a.uniform && prob[0] > 0.f) {
-      float total = 0.f;
-      for (int i = 0; i < k; ++i) total += prob[i];
-      const float target = a.uniform[row] * total;
-      float cum = 0.f;
-      pick = -1;
-      for (int i = 0; i < k; ++i) {
-        if (prob[i] == 0.f) continue;
-        cum += prob[i];
-        pick = i;
-        if (cum > target) break;
+  if (tid < 32 && a.token) {
+    // inverse CDF over the k (<= 64) survivors in rank order: warp 0 holds
+    // survivors lane and lane + 32 and scans their probabilities; the draw is
+    // the first survivor (p > 0) whose cumulative sum exceeds u * total, else
+    // the last one with p > 0
+    const int lane = tid;
+    const float p_lo = lane < k ? prob[lane] : 0.f;
+    const float p_hi = lane + 32 < k ? prob[lane + 32] : 0.f;
+    float c_lo = p_lo, c_hi = p_hi;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y_lo = __shfl_up_sync(0xffffffffu, c_lo, off);
+      const float y_hi = __shfl_up_sync(0xffffffffu, c_hi, off);
+      if (lane >= off) {
+        c_lo += y_lo;
+        c_hi += y_hi;
       }
     }
-    a.token[row] = (int)(0xFFFFFFFFu - (uint32_t)sorted[pick]);
+    c_hi += __shfl_sync(0xffffffffu, c_lo, 31);
+    const float total = __shfl_sync(0xffffffffu, c_hi, 31);
+    int pick = 0;
+    if (a.uniform && prob[0] > 0.f) {
+      const float target = a.uniform[row] * total;
+      const uint32_t over_lo = __ballot_sync(0xffffffffu, p_lo > 0.f && c_lo > target);
+      const uint32_t over_hi = __ballot_sync(0xffffffffu, p_hi > 0.f && c_hi > target);
+      const uint32_t pos_lo = __ballot_sync(0xffffffffu, p_lo > 0.f);
+      const uint32_t pos_hi = __ballot_sync(0xffffffffu, p_hi > 0.f);
+      if (over_lo) pick = __ffs(over_lo) - 1;
+      else if (over_hi) pick = 32 + __ffs(over_hi) - 1;
+      else pick = pos_hi ? 63 - __clz(pos_hi) : 31 - __clz(pos_lo);
+    }
+    if (lane == 0) a.token[row] = (int)(0xFFFFFFFFu - (uint32_t)sorted[pick]);
   }
 }
 
