@@ -337,30 +337,36 @@ __global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs/SM: 64 rows x 8 CTAs i
 // logits mostly share sign and exponent) over the bins from the first pass,
 // so the histogram atomics rarely collide.  CTA-wide; keys in shared memory;
 // ends with a barrier.
+// (smallest, largest) of the keys: span[i] and span[kSpanHalf + i] for
+// i < nspan hold partial minima and maxima already (nspan > 0), or the CTA
+// works them out here (nspan = 0).
+constexpr int kSpanHalf = kMaxTopkCluster > kWarps ? kMaxTopkCluster : kWarps;
 __device__ unsigned long long cta_kth_threshold(const unsigned long long *keys, int n, int k,
                                                 uint32_t *hist, uint32_t *scan, uint32_t *sel,
-                                                unsigned long long *span) {
+                                                unsigned long long *span, int nspan) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  unsigned long long lo = ~0ull, hi = 0;
-  for (int i = tid; i < n; i += kThreads) {
-    lo = min(lo, keys[i]);
-    hi = max(hi, keys[i]);
-  }
+  if (nspan == 0) {
+    unsigned long long lo = ~0ull, hi = 0;
+    for (int i = tid; i < n; i += kThreads) {
+      lo = min(lo, keys[i]);
+      hi = max(hi, keys[i]);
+    }
 #pragma unroll
-  for (int off = 16; off; off >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    for (int off = 16; off; off >>= 1) {
+      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+      span[warp] = lo;
+      span[kSpanHalf + warp] = hi;
+    }
+    nspan = kWarps;
+    __syncthreads();
   }
-  if (lane == 0) {  // span: 2 x kWarps
-    span[warp] = lo;
-    span[kWarps + warp] = hi;
-  }
-  __syncthreads();
-  lo = span[0];
-  hi = span[kWarps];
-  for (int i = 1; i < kWarps; ++i) {
+  unsigned long long lo = span[0], hi = span[kSpanHalf];
+  for (int i = 1; i < nspan; ++i) {
     lo = min(lo, span[i]);
-    hi = max(hi, span[kWarps + i]);
+    hi = max(hi, span[kSpanHalf + i]);
   }
   if (lo == hi) {
     __syncthreads();  // span is rewritten by the next call
@@ -428,7 +434,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan[kWarps];
   __shared__ uint32_t sel[3];
-  __shared__ unsigned long long span[2 * kWarps];
+  __shared__ unsigned long long span[2 * kSpanHalf];  // leader: the CTAs' (min, max) thread maxima
+  __shared__ unsigned long long wspan[2 * kWarps];
   __shared__ unsigned long long thr;               // T, written by the leader into every CTA
   __shared__ uint32_t n_cand, n_top;               // leader: candidates received, selected
   __shared__ unsigned long long sorted[kTopkMax];
@@ -463,10 +470,32 @@ __global__ void __launch_bounds__(kThreads, 4)
   // ---- 2. thread maxima into the leader; T back to every CTA
   cluster_wait_acquire();  // every CTA of the cluster has started
   st_cluster_u64(map_to_rank(&keybuf[rank * kThreads + tid], 0), key);
+  {
+    // this CTA's smallest and largest thread maximum, for the leader's select
+    unsigned long long mn = key, mx = key;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    if ((tid & 31) == 0) {
+      wspan[tid >> 5] = mn;
+      wspan[kWarps + (tid >> 5)] = mx;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < kWarps; ++w) {
+        mn = min(mn, wspan[w]);
+        mx = max(mx, wspan[kWarps + w]);
+      }
+      st_cluster_u64(map_to_rank(&span[rank], 0), mn);
+      st_cluster_u64(map_to_rank(&span[kSpanHalf + rank], 0), mx);
+    }
+  }
   cluster_arrive_release();
   cluster_wait_acquire();
   if (rank == 0) {
-    const unsigned long long T = cta_kth_threshold(keybuf, C * kThreads, a.k, hist, scan, sel, span);
+    const unsigned long long T = cta_kth_threshold(keybuf, C * kThreads, a.k, hist, scan, sel, span, C);
     if (tid < C) st_cluster_u64(map_to_rank(&thr, tid), T);
   }
   cluster_arrive_release();
@@ -531,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     __syncthreads();
   } else {
-    const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel, span);
+    const unsigned long long T2 = cta_kth_threshold(keybuf, nc, k, hist, scan, sel, span, 0);
     for (int i = tid; i < nc; i += kThreads) {
       const unsigned long long kk = keybuf[i];
       if (kk >= T2) {
