@@ -9,8 +9,9 @@
 // One CTA computes two consecutive 128-row query tiles A = 2i and B = 2i + 1
 // of one (sequence, head); both read every K/V tile they need once from
 // shared memory:
-//   warp 8      TMA producer: Q_A and Q_B once, then K and V tiles (128 keys x
-//               128 dims, bf16, 128-byte swizzle) into a 2-stage ring;
+//   warp 8      TMA producer: Q_A and Q_B once, then K tiles (128 keys x 128
+//               dims, bf16, 128-byte swizzle) into a 2-stage ring;
+//   warp 10     TMA producer of the V tiles (3-stage ring);
 //   warp 9      MMA issuer (one thread) and TMEM owner (512 columns:
 //               S_A, S_B, O_A, O_B, 128 fp32 columns each).  Order per key
 //               tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so each softmax
@@ -24,6 +25,8 @@
 //               warp's running max grows by more than 2^8; otherwise the stale
 //               max keeps every p <= 256, exact in the end because l uses the
 //               same max.  The epilogue divides by l and stores bf16 rows.
+// Warps 8-11 (warp 11 has no role) hand registers to the softmax warpgroups
+// (setmaxnreg), which hold a whole 128-score row per thread.
 // Blocks are grouped by (sequence, head), longest first inside a group, so
 // the CTAs running together share their K/V tiles through L2.  Every mbarrier
 // wait is bounded; on a timeout the kernel records it, stops issuing work,
