@@ -27,7 +27,8 @@
 //    CTA's column range is requested into L2 by bulk prefetches at kernel
 //    start, so the row leaves DRAM at full depth.
 //  - k > 1: the leader gathers the C x 256 thread maxima and finds their k-th
-//    largest, T, by a CTA-local radix select (8 bits per pass).  At least k
+//    largest, T, by a CTA-local radix select (8 bits per pass, over the keys'
+//    offsets from the smallest of them).  At least k
 //    keys of the row are >= T, and they all lie in the k threads whose
 //    maximum is >= T.  A thread whose second largest key is known and below T
 //    sends only its maximum; the others with a maximum >= T reread their
@@ -148,8 +149,8 @@ __device__ void reject_row(const TopkArgs &a, int row, int rank) {
 // CTA's whole range is first requested into L2 by bulk prefetches, so the
 // row streams from DRAM at full depth) and keeps the two first
 // maxima of them in increasing column order; the ban is worked out while the
-// last two batches are in flight (the history was copied asynchronously at
-// the start).  If a thread's best is banned its second is the answer, unless
+// last two batches are in flight (top-1 form) or right after the stream
+// (top-k form); the history was copied asynchronously at the start.  If a thread's best is banned its second is the answer, unless
 // that is banned too, in which case the thread rescans its columns (from L2)
 // skipping banned ones -- which needs two banned tokens among one thread's 64
 // columns.  Returns the thread's largest masked key ((order image of the
@@ -225,10 +226,20 @@ __device__ __forceinline__ unsigned long long stream_thread_max(const TopkArgs &
   load_batch(x0, 2 * kBatch);
   consume(x1, kBatch);
   load_batch(x1, 3 * kBatch);
-  *bad = ban_prologue(a, row, col0, ban_bits, hist_s);
-  if (*bad) return 0;
+  // The ban's barriers hold every warp of the CTA.  The top-1 form works it
+  // out while its last two batches are in flight (10.7 against 11.2 us per
+  // call with it after the stream); the top-k form, which has a second pass
+  // behind it, after the stream (20.45 against 20.7 us).
+  if (kEvictFirst) {
+    *bad = ban_prologue(a, row, col0, ban_bits, hist_s);
+    if (*bad) return 0;
+  }
   consume(x0, 2 * kBatch);
   consume(x1, 3 * kBatch);
+  if (!kEvictFirst) {
+    *bad = ban_prologue(a, row, col0, ban_bits, hist_s);
+    if (*bad) return 0;
+  }
 
   const auto banned = [&](int col) {
     const int f = col - col0;
