@@ -71,6 +71,47 @@ def test_rope_prefill_and_decode_vs_oracle(policy, dtype, d, split, monkeypatch)
     assert st.check() == 0
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("policy", ["absolute", "slot"])
+def test_rope_long_prompt_sampled_rows_and_ring_wrap(policy):
+    """A 32,640-token prompt (the near-max length): rotation angles up to
+    ~3.3e4 radians, where the reduction of the angle matters.  Sampled query
+    rows of the prefill against the oracle, sampled rotated cache rows within
+    one bf16 rounding, then W + 3 decode steps (one ring wrap) step by step."""
+    from ring_sliding_window_b200 import rswa
+    B, L, H, d, W, theta = 1, 1, 2, 128, 128, 10000.0
+    P = (32640,)
+    w = synth.Workload("rope_long", 62, torch.bfloat16, B, L, H, d, W, P, W + 3)
+    st = rswa.State(B, L, H, d, W, P, dtype=torch.bfloat16)
+    st.set_rope(POLICIES[policy], theta)
+    tol = tol_for(torch.bfloat16)
+    q, k, v = synth.prefill_qkv(w, 0, "cuda")
+    out = torch.empty_like(q)
+    st.prefill(0, q, k, v, out)
+    pos = np.arange(P[0])
+    qr, kr, vv = oracle.rope(f64(q), pos, theta), oracle.rope(f64(k), pos, theta), f64(v)
+    for r in (0, 1, 127, 128, 4095, 16383, 16384, 32511, 32639):
+        ref = oracle.prefill(qr[:r + 1], kr[:r + 1], vv[:r + 1], w.scale, r, r + 1)[r]
+        assert np.max(np.abs(f64(out[r]) - ref)) <= tol, r
+    rows = np.array([0, 1, 8191, 16384, 30000, 32639])
+    for h in range(H):
+        gk = f64(st.cache_view(0, "k", 0, h)[rows])
+        assert np.all(np.abs(gk - kr[rows, h]) <= 2.0 ** -8 * np.abs(kr[rows, h]) + 1e-6), h
+    model = oracle.RingModel(P, W, L, H, d)
+    model.prefill(0, 0, kr, vv)
+    for t in range(W + 3):
+        qd, kn, vn = synth.decode_qkv(w, 0, t, "cuda")
+        o = torch.empty_like(qd)
+        st.decode_step(0, qd, kn, vn, o)
+        p = [oracle.rope_position(policy, P[0], t, W)]
+        ref, _, _ = model.rings[0][0].step(oracle.rope(f64(qd[0])[None], p, theta)[0],
+                                           oracle.rope(f64(kn[0])[None], p, theta)[0],
+                                           f64(vn[0]), w.scale)
+        assert np.max(np.abs(f64(o[0]) - ref)) <= tol, t
+        st.advance()
+    assert st.check() == 0
+
+
 def test_rope_reset_and_policy_errors():
     from ring_sliding_window_b200 import rswa
     st = rswa.State(1, 1, 2, 128, 8, [64], dtype=torch.bfloat16)
