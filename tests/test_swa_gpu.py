@@ -70,6 +70,30 @@ def test_standard_swa_prefill_and_decode(dtype, d, split, W, monkeypatch):
     assert st.check() == 0
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("W", [128, 300])
+def test_standard_swa_long_prompt_sampled_rows(W):
+    """An 8,256-token prompt (the multi-page length) in standard-SWA mode:
+    every query tile reads only the key tiles of its window.  Sampled rows at
+    tile and window boundaries against the windowed attention of the oracle."""
+    from ring_sliding_window_b200 import rswa
+    B, L, H, d = 1, 1, 2, 128
+    P = (8256,)
+    w = synth.Workload("swa_long", 75, torch.bfloat16, B, L, H, d, W, P, 0)
+    st = rswa.State(B, L, H, d, W, P, dtype=torch.bfloat16)
+    st.set_attention(rswa.RSWA_ATTN_STANDARD_SWA)
+    q, k, v = synth.prefill_qkv(w, 0, "cuda")
+    out = torch.empty_like(q)
+    st.prefill(0, q, k, v, out)
+    qq, kk, vv, oo = f64(q), f64(k), f64(v), f64(out)
+    for i in (0, 1, 127, 128, W - 1, W, 255, 256, 300, 4000, 8063, 8064, 8191, 8192, 8255):
+        lo = max(0, i - W + 1)
+        for h in range(H):
+            ref = oracle.attend(qq[i, h], kk[lo:i + 1, h], vv[lo:i + 1, h], w.scale)
+            assert np.max(np.abs(oo[i, h] - ref)) <= tol_for(torch.bfloat16), (i, h)
+    assert st.check() == 0
+
+
 def test_attention_mode_switch_and_errors():
     from ring_sliding_window_b200 import rswa
     st = rswa.State(1, 1, 2, 128, 8, [64], dtype=torch.bfloat16)
