@@ -65,6 +65,46 @@ def test_keysplit_shares_vs_oracle(shares, split, dtype, d, monkeypatch):
         st.close()
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("shares", [2, 4])
+def test_keysplit_near_max_length_across_a_ring_wrap(shares):
+    """The near-max sequence (32,640 prompt tokens, 10 heads x 128, W = 128)
+    split over 2 and 4 shares, W + 2 decode steps (one ring wrap), every step
+    against the FP64 ring oracle over the whole cache."""
+    from ring_sliding_window_b200 import rswa
+    from ring_sliding_window_b200.keysplit import share_bounds
+    H, d, W, P, L = 10, 128, 128, 32640, 1
+    steps = W + 2
+    w = synth.Workload("keysplit_long", 83, torch.bfloat16, 1, L, H, d, W, (P,), steps)
+    q, k, v = synth.prefill_qkv(w, 0, "cuda")
+    model = oracle.RingModel((P,), W, L, H, d)
+    model.prefill(0, 0, f64(k), f64(v))
+    bounds = share_bounds(P, shares)
+    states = []
+    for lo, hi in bounds:
+        st = rswa.State(1, L, H, d, W, [hi - lo], dtype=torch.bfloat16)
+        st.prefill(0, q[lo:hi], k[lo:hi], v[lo:hi], torch.empty_like(q[lo:hi]))
+        states.append(st)
+    del q, k, v
+    ml = torch.empty(shares, 1, H, 2, dtype=torch.float32, device="cuda")
+    o = torch.empty(shares, 1, H, d, dtype=torch.float32, device="cuda")
+    for t in range(steps):
+        qs, kn, vn = synth.decode_qkv(w, 0, t, "cuda")
+        for g, st in enumerate(states):
+            lo, hi = bounds[g]
+            key_hi = (hi - lo) + (W if g == shares - 1 else 0)
+            st.decode_step_partial(0, qs, kn, vn, 0, key_hi, ml[g], o[g])
+        out = torch.empty_like(qs)
+        rswa.rswa_combine_partials(ml, o, out)
+        ref = model.step(0, f64(qs), f64(kn), f64(vn), w.scale)
+        assert np.max(np.abs(f64(out) - ref)) <= tol_for(torch.bfloat16), t
+        for st in states:
+            st.advance()
+    for st in states:
+        assert st.check() == 0
+        st.close()
+
+
 def test_partial_ranges_of_one_state_match_the_full_step():
     """Two calls over [0, a) and [a, end) of the same state merge to the
     output of rswa_decode_step (the second call performs the ring write)."""
