@@ -114,3 +114,70 @@ def test_continuous_batching_vs_oracle(dtype, d, split, monkeypatch):
     assert expect_base["A"] == 0 and expect_base["D"] == 0
     assert expect_base["E"] == 68 and expect_base["F"] == 106
     pool.close()
+
+
+@pytest.mark.slow
+def test_continuous_batching_serving_sizes():
+    """Ragged-serving sizes on one pool: 8 requests with prompts of 1,024 to
+    16,384 tokens, W = 128, 10 heads x 128; 2 leave and 2 join at step 60 (the
+    joiners land in freed ranges) and again at step 133, after the first
+    requests' rings have wrapped.  Every step's outputs against the oracle;
+    every live cache bit-exact at the end."""
+    from ring_sliding_window_b200 import rswa
+    L, H, d, W, steps = 1, 10, 128, 128, 140
+    dtype = torch.bfloat16
+    scale = 1.0 / np.sqrt(d)
+    rng = np.random.default_rng(7)
+    plen = {i: int(rng.integers(1024, 16385)) for i in range(12)}
+    schedule = {0: ([], list(range(8))), 60: ([1, 5], [8, 9]), 133: ([0, 8], [10, 11])}
+    capacity = int(1.25 * sum(plen[i] + W for i in range(8))) + 2 * (16384 + W)
+    pool = rswa.TokenPool(capacity, L, H, d, W, dtype=dtype)
+    seed = lambda req, step, what: synth.seed(90 + req, 0, 3 * step + what)  # noqa: E731
+    live, st = [], None
+    for step in range(steps):
+        leaving, joining = schedule.get(step, ([], []))
+        if leaving or joining:
+            if st is not None:
+                st.close()
+            for rid in leaving:
+                r = next(r for r in live if r["id"] == rid)
+                pool.free(r["base"])
+                live.remove(r)
+            new = []
+            for rid in joining:
+                P = plen[rid]
+                new.append({"id": rid, "P": P, "base": pool.alloc(P), "t": 0,
+                            "ring": oracle.Ring(P, W, H, d)})
+            pst = pool.state([r["P"] for r in new], [r["base"] for r in new])
+            ks, vs = [], []
+            for r in new:
+                ks.append(synth.normal((r["P"], H, d), seed(r["id"], 10_000, 0), dtype, "cuda"))
+                vs.append(synth.normal((r["P"], H, d), seed(r["id"], 10_000, 1), dtype, "cuda"))
+                r["ring"].prefill(f64(ks[-1]), f64(vs[-1]))
+            k, v = torch.cat(ks), torch.cat(vs)
+            pst.prefill(0, torch.zeros_like(k), k, v, torch.empty_like(k))
+            pst.close()
+            del k, v, ks, vs
+            live.extend(new)
+            st = pool.state([r["P"] for r in live], [r["base"] for r in live],
+                            n_generated=[r["t"] for r in live])
+        q, kn, vn = (torch.stack([synth.normal((H, d), seed(r["id"], step, i), dtype, "cuda")
+                                  for r in live]) for i in range(3))
+        out = torch.empty_like(q)
+        st.decode_step(0, q, kn, vn, out)
+        for b, r in enumerate(live):
+            ref, _, _ = r["ring"].step(f64(q[b]), f64(kn[b]), f64(vn[b]), scale)
+            assert np.max(np.abs(f64(out[b]) - ref)) <= tol_for(dtype), (step, r["id"])
+        st.advance()
+        for r in live:
+            r["t"] += 1
+    n, _, _ = st.ring()
+    assert n == [r["t"] for r in live]
+    for b, r in enumerate(live):
+        kc, vc, held = r["ring"].snapshot()
+        for h in range(H):
+            assert np.array_equal(f64(st.cache_view(0, "k", b, h)[:held]), kc[:held, h])
+            assert np.array_equal(f64(st.cache_view(0, "v", b, h)[:held]), vc[:held, h])
+    assert st.check() == 0
+    st.close()
+    pool.close()
