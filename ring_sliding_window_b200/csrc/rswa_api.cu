@@ -145,7 +145,16 @@ std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen,
   for (int b = 0; b < B; ++b) {
     const int tiles = (int)((plen[b] + kPrefillTile - 1) / kPrefillTile);
     for (int h = 0; h < H; ++h) {
-      for (int t0 = 0; t0 < tiles; t0 += per_block)
+      // With an odd tile count one tile has no partner, and a lone tile runs
+      // at about half the rate of a pair (its softmax has no other tile's
+      // MMAs to overlap).  Make that tile the first, whose single key tile
+      // costs little, so the last, longest tiles are paired.
+      int t0 = 0;
+      if (per_block == 2 && (tiles & 1)) {
+        group.push_back(make_int4(b, h, 0, 1));
+        t0 = 1;
+      }
+      for (; t0 < tiles; t0 += per_block)
         group.push_back(make_int4(b, h, t0, tiles - t0 >= per_block ? per_block : 1));
       group_blocks += (tiles + per_block - 1) / per_block;
       if (group_blocks >= num_sms) flush();
