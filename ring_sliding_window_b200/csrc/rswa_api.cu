@@ -133,8 +133,13 @@ std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen,
   for (int b = 0; b < B; ++b) pairs += (int64_t)H * ((plen[b] + 2 * kPrefillTile - 1) / (2 * kPrefillTile));
   const int per_block = pairs >= num_sms && !one_tile ? 2 : 1;
   std::vector<int4> out;
-  std::vector<int4> group;
+  std::vector<int4> group, tail;
   int64_t group_blocks = 0;
+  // A batch of several waves ends with the blocks of short query tiles (the
+  // first eighth of every prompt's tiles), longest first: the last wave then
+  // holds no long block that the other SMs would wait for.  Those blocks read
+  // few K/V tiles, so losing their L2 sharing costs little.
+  const bool defer = per_block == 2 && pairs >= 4 * (int64_t)num_sms;
   auto flush = [&]() {
     std::stable_sort(group.begin(), group.end(),
                      [](const int4 &x, const int4 &y) { return x.z > y.z; });
@@ -154,13 +159,21 @@ std::vector<int4> plan_prefill_blocks(const rswa_config *c, const int64_t *plen,
         group.push_back(make_int4(b, h, 0, 1));
         t0 = 1;
       }
-      for (; t0 < tiles; t0 += per_block)
-        group.push_back(make_int4(b, h, t0, tiles - t0 >= per_block ? per_block : 1));
+      for (; t0 < tiles; t0 += per_block) {
+        const int4 blk = make_int4(b, h, t0, tiles - t0 >= per_block ? per_block : 1);
+        if (defer && t0 < tiles / 8)
+          tail.push_back(blk);
+        else
+          group.push_back(blk);
+      }
       group_blocks += (tiles + per_block - 1) / per_block;
       if (group_blocks >= num_sms) flush();
     }
   }
   flush();
+  std::stable_sort(tail.begin(), tail.end(),
+                   [](const int4 &x, const int4 &y) { return x.z > y.z; });
+  out.insert(out.end(), tail.begin(), tail.end());
   return out;
 }
 
