@@ -6,9 +6,9 @@
 // transformers path materialises the whole score matrix; here it is a
 // flash-style kernel that never leaves the chip with it.
 //
-// One CTA computes two consecutive 128-row query tiles A = 2i and B = 2i + 1
-// of one (sequence, head); both read every K/V tile they need once from
-// shared memory:
+// One CTA computes two consecutive 128-row query tiles A and B = A + 1 of one
+// (sequence, head); both read every K/V tile they need once from shared
+// memory:
 //   warp 8      TMA producer: Q_A and Q_B once, then K tiles (128 keys x 128
 //               dims, bf16, 128-byte swizzle) into a 2-stage ring;
 //   warp 10     TMA producer of the V tiles (3-stage ring);
@@ -198,129 +198,129 @@ __global__ void __launch_bounds__(kThreads, 1)
   // at the top of its own branch, so the compiler allocates each branch
   // within its own count.
   if (warp >= 8) {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kAuxRegs));
-  if (warp == kProducerWarp || warp == kVProducerWarp) {
-    // ------------------------------------------------------------ producers
-    // warp 8 loads Q and the K ring, warp 10 the V ring, so a K load never
-    // waits behind a V slot that is still in use (and the other way round).
-    if (lane == 0) {
-      const bool is_k = warp == kProducerWarp;
-      // test-only fault injection: no loads at all, so every wait on them
-      // runs out (bounded) and the kernel takes its timeout path
-      const bool drop_loads = (*v.fault & RSWA_FAULT_DROP_PREFILL_LOADS) != 0;
-      const int xh = h * kD;
-      const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
-      const int nst = is_k ? kKStages : kVStages;
-      tc::prefetch_tmap(tm);
-      if (is_k && !drop_loads) {
-        tc::prefetch_tmap(&tm_q);
-        mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(ntiles * kTileBytes));
-        for (int x = 0; x < ntiles; ++x) {
-          const int y = tok0 + (qt0 + x) * kTile;
-          tc::tma_load_2d(sm.q[x], &tm_q, xh, y, &sm.q_full);
-          tc::tma_load_2d(sm.q[x] + kHalfBytes, &tm_q, xh + 64, y, &sm.q_full);
-        }
-      }
-      int issued = 0;
-      // K from the cache: rows H * S_b + h * (P_b + W) + key of a [rows][128]
-      // map (rows past the prompt are ring slots: masked, like the causal
-      // overhang of the input layout)
-      const bool from_cache = is_k && a.k_from_cache;
-      const int x0 = from_cache ? 0 : xh;
-      const int y0 = from_cache ? (int)((int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W))
-                                : tok0;
-      for (int j = 0; !drop_loads && j < n_kv_all; ++j) {
-        const int s = j % nst;
-        uint64_t *empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
-        uint64_t *full = is_k ? &sm.k_full[s] : &sm.v_full[s];
-        uint8_t *dst = is_k ? sm.k[s] : sm.v[s];
-        if (!wait_bar(empty, ((j / nst) & 1) ^ 1, v.err, dead)) break;
-        mbar_arrive_expect_tx(full, kTileBytes);
-        tc::tma_load_2d(dst, tm, x0, y0 + (j0 + j) * kTile, full);
-        tc::tma_load_2d(dst + kHalfBytes, tm, x0 + 64, y0 + (j0 + j) * kTile, full);
-        issued = j + 1;
-      }
-      // every load issued has landed before the CTA may exit (bounded)
-      if (is_k && !drop_loads) mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
-      for (int s = 0; s < nst && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / nst) * nst;
-        mbar_wait_bounded(is_k ? &sm.k_full[s] : &sm.v_full[s], (last / nst) & 1, v.err,
-                          RSWA_DEVERR_TIMEOUT);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t q_addr0 = smem_u32(sm.q[0]);
-      // key tile j0 + it lands in K slot it mod 2 / V slot it mod 3; send it to
-      // the cache if it is one of this block's whole prompt tiles
-      bool stored = false;
-      auto store_tile = [&](const CUtensorMap *tm, const uint8_t *src, int it) {
-        const int kt = j0 + it;
-        if (kt < qt0 || kt >= n_full_tiles) return;
-        const int y = (int)(crow0 + (int64_t)kt * kTile);
-        tc::tma_store_2d(tm, src, 0, y);
-        tc::tma_store_2d(tm, src + kHalfBytes, 64, y);
-        stored = true;
-      };
-      bool ok = wait_bar(&sm.q_full, 0, v.err, dead) &&
-                wait_bar(&sm.k_full[0], 0, v.err, dead);
-      if (ok) {
-        tc::fence_after_sync();
-        if (a.store_k) store_tile(&tm_kc, sm.k[0], 0);
-        for (int x = 0; x < ntiles; ++x) {
-          issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[0]));
-          tc::commit(&sm.s_full[x]);
-        }
-        tc::commit(&sm.k_empty[0]);
-      }
-      for (int j = 0; ok && j < n_kv_all; ++j) {
-        const int s = j % kVStages;          // V stage of tile j
-        const int s1 = (j + 1) % kKStages;   // K stage of tile j + 1
-        bool k1_ready = false;  // K_{j+1} waited for
-        if (!(ok = wait_bar(&sm.v_full[s], (j / kVStages) & 1, v.err, dead))) break;
-        if (a.store_v) store_tile(&tm_vc, sm.v[s], j);
-        // K_{j+1} has usually landed by now: taking it here keeps the barrier
-        // check out of the gap between P V and the next Q K^T of tile A (a
-        // wait issued right after a burst of MMAs costs 50-200 cycles).  If
-        // it has not, it is waited for there, as before.
-        if (j + 1 < n_kv_all && mbar_try_wait(&sm.k_full[s1], ((j + 1) / kKStages) & 1)) {
-          tc::fence_after_sync();
-          k1_ready = true;
-          if (a.store_k) store_tile(&tm_kc, sm.k[s1], j + 1);
-        }
-        for (int x = 0; x < ntiles; ++x) {
-          const int nkv = x == 0 ? n_kv_a : n_kv_b;
-          if (j >= nkv) continue;
-          // O_X += P_X(j) V_j
-          if (!(ok = wait_bar(&sm.p_full[x], j & 1, v.err, dead))) break;
-          tc::fence_after_sync();
-          issue_pv(tbase + col_o(x), tbase + col_s(x), smem_u32(sm.v[s]), j > 0);
-          if (j == nkv - 1) tc::commit(&sm.o_final[x]);
-          // S_X(j+1) = Q_X K_{j+1}^T  (overwrites P_X(j): issued after PV_X(j))
-          if (j + 1 < nkv) {
-            if (!k1_ready) {
-              if (!(ok = wait_bar(&sm.k_full[s1], ((j + 1) / kKStages) & 1, v.err, dead))) break;
-              tc::fence_after_sync();
-              k1_ready = true;
-              if (a.store_k) store_tile(&tm_kc, sm.k[s1], j + 1);
-            }
-            issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[s1]));
-            tc::commit(&sm.s_full[x]);
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kAuxRegs));
+    if (warp == kProducerWarp || warp == kVProducerWarp) {
+      // ------------------------------------------------------------ producers
+      // warp 8 loads Q and the K ring, warp 10 the V ring, so a K load never
+      // waits behind a V slot that is still in use (and the other way round).
+      if (lane == 0) {
+        const bool is_k = warp == kProducerWarp;
+        // test-only fault injection: no loads at all, so every wait on them
+        // runs out (bounded) and the kernel takes its timeout path
+        const bool drop_loads = (*v.fault & RSWA_FAULT_DROP_PREFILL_LOADS) != 0;
+        const int xh = h * kD;
+        const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+        const int nst = is_k ? kKStages : kVStages;
+        tc::prefetch_tmap(tm);
+        if (is_k && !drop_loads) {
+          tc::prefetch_tmap(&tm_q);
+          mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(ntiles * kTileBytes));
+          for (int x = 0; x < ntiles; ++x) {
+            const int y = tok0 + (qt0 + x) * kTile;
+            tc::tma_load_2d(sm.q[x], &tm_q, xh, y, &sm.q_full);
+            tc::tma_load_2d(sm.q[x] + kHalfBytes, &tm_q, xh + 64, y, &sm.q_full);
           }
         }
-        if (!ok) break;
-        tc::commit(&sm.v_empty[s]);
-        if (k1_ready) tc::commit(&sm.k_empty[s1]);
+        int issued = 0;
+        // K from the cache: rows H * S_b + h * (P_b + W) + key of a [rows][128]
+        // map (rows past the prompt are ring slots: masked, like the causal
+        // overhang of the input layout)
+        const bool from_cache = is_k && a.k_from_cache;
+        const int x0 = from_cache ? 0 : xh;
+        const int y0 = from_cache ? (int)((int64_t)v.H * v.slot_base[b] + (int64_t)h * (P + v.W))
+                                  : tok0;
+        for (int j = 0; !drop_loads && j < n_kv_all; ++j) {
+          const int s = j % nst;
+          uint64_t *empty = is_k ? &sm.k_empty[s] : &sm.v_empty[s];
+          uint64_t *full = is_k ? &sm.k_full[s] : &sm.v_full[s];
+          uint8_t *dst = is_k ? sm.k[s] : sm.v[s];
+          if (!wait_bar(empty, ((j / nst) & 1) ^ 1, v.err, dead)) break;
+          mbar_arrive_expect_tx(full, kTileBytes);
+          tc::tma_load_2d(dst, tm, x0, y0 + (j0 + j) * kTile, full);
+          tc::tma_load_2d(dst + kHalfBytes, tm, x0 + 64, y0 + (j0 + j) * kTile, full);
+          issued = j + 1;
+        }
+        // every load issued has landed before the CTA may exit (bounded)
+        if (is_k && !drop_loads) mbar_wait_bounded(&sm.q_full, 0, v.err, RSWA_DEVERR_TIMEOUT);
+        for (int s = 0; s < nst && s < issued; ++s) {
+          const int last = s + ((issued - 1 - s) / nst) * nst;
+          mbar_wait_bounded(is_k ? &sm.k_full[s] : &sm.v_full[s], (last / nst) & 1, v.err,
+                            RSWA_DEVERR_TIMEOUT);
+        }
       }
-      tc::commit(&sm.mma_done);
-      if (stored) {
-        tc::store_commit();
-        tc::store_wait_read();  // the tiles stay in shared memory until read
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t q_addr0 = smem_u32(sm.q[0]);
+        // key tile j0 + it lands in K slot it mod 2 / V slot it mod 3; send it to
+        // the cache if it is one of this block's whole prompt tiles
+        bool stored = false;
+        auto store_tile = [&](const CUtensorMap *tm, const uint8_t *src, int it) {
+          const int kt = j0 + it;
+          if (kt < qt0 || kt >= n_full_tiles) return;
+          const int y = (int)(crow0 + (int64_t)kt * kTile);
+          tc::tma_store_2d(tm, src, 0, y);
+          tc::tma_store_2d(tm, src + kHalfBytes, 64, y);
+          stored = true;
+        };
+        bool ok = wait_bar(&sm.q_full, 0, v.err, dead) &&
+                  wait_bar(&sm.k_full[0], 0, v.err, dead);
+        if (ok) {
+          tc::fence_after_sync();
+          if (a.store_k) store_tile(&tm_kc, sm.k[0], 0);
+          for (int x = 0; x < ntiles; ++x) {
+            issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[0]));
+            tc::commit(&sm.s_full[x]);
+          }
+          tc::commit(&sm.k_empty[0]);
+        }
+        for (int j = 0; ok && j < n_kv_all; ++j) {
+          const int s = j % kVStages;          // V stage of tile j
+          const int s1 = (j + 1) % kKStages;   // K stage of tile j + 1
+          bool k1_ready = false;  // K_{j+1} waited for
+          if (!(ok = wait_bar(&sm.v_full[s], (j / kVStages) & 1, v.err, dead))) break;
+          if (a.store_v) store_tile(&tm_vc, sm.v[s], j);
+          // K_{j+1} has usually landed by now: taking it here keeps the barrier
+          // check out of the gap between P V and the next Q K^T of tile A (a
+          // wait issued right after a burst of MMAs costs 50-200 cycles).  If
+          // it has not, it is waited for there, as before.
+          if (j + 1 < n_kv_all && mbar_try_wait(&sm.k_full[s1], ((j + 1) / kKStages) & 1)) {
+            tc::fence_after_sync();
+            k1_ready = true;
+            if (a.store_k) store_tile(&tm_kc, sm.k[s1], j + 1);
+          }
+          for (int x = 0; x < ntiles; ++x) {
+            const int nkv = x == 0 ? n_kv_a : n_kv_b;
+            if (j >= nkv) continue;
+            // O_X += P_X(j) V_j
+            if (!(ok = wait_bar(&sm.p_full[x], j & 1, v.err, dead))) break;
+            tc::fence_after_sync();
+            issue_pv(tbase + col_o(x), tbase + col_s(x), smem_u32(sm.v[s]), j > 0);
+            if (j == nkv - 1) tc::commit(&sm.o_final[x]);
+            // S_X(j+1) = Q_X K_{j+1}^T  (overwrites P_X(j): issued after PV_X(j))
+            if (j + 1 < nkv) {
+              if (!k1_ready) {
+                if (!(ok = wait_bar(&sm.k_full[s1], ((j + 1) / kKStages) & 1, v.err, dead))) break;
+                tc::fence_after_sync();
+                k1_ready = true;
+                if (a.store_k) store_tile(&tm_kc, sm.k[s1], j + 1);
+              }
+              issue_qk(tbase + col_s(x), q_addr0 + (uint32_t)x * kTileBytes, smem_u32(sm.k[s1]));
+              tc::commit(&sm.s_full[x]);
+            }
+          }
+          if (!ok) break;
+          tc::commit(&sm.v_empty[s]);
+          if (k1_ready) tc::commit(&sm.k_empty[s1]);
+        }
+        tc::commit(&sm.mma_done);
+        if (stored) {
+          tc::store_commit();
+          tc::store_wait_read();  // the tiles stay in shared memory until read
+        }
+        mbar_wait_bounded(&sm.mma_done, 0, v.err, RSWA_DEVERR_TIMEOUT);
       }
-      mbar_wait_bounded(&sm.mma_done, 0, v.err, RSWA_DEVERR_TIMEOUT);
     }
-  }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ------------------------------------------------------------ softmax
