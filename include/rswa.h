@@ -470,6 +470,16 @@ rswa_status rswa_decode_step_noalloc(const rswa_config *cfg, const int64_t *pref
 #define RSWA_FAULT_DROP_PREFILL_LOADS 2
 rswa_status rswa_debug_inject_fault(rswa_state *state, int32_t flags, void *stream);
 
+/* ---- Prefill work plan (tests only) ---------------------------------------
+ * The blocks the tensor-core prefill (bf16, d = 128) would launch for this
+ * batch on a part with `num_sms` SMs, in launch order: 4 int32 per block,
+ * (request b, head h, first query tile, query tiles 1 or 2), into `out`
+ * (host, room for `capacity` blocks).  Host only: no device is touched.
+ * Returns the number of blocks (those past `capacity` are not written), or
+ * -1 for a bad config or arguments. */
+int64_t rswa_debug_prefill_plan(const rswa_config *cfg, const int64_t *prefill_len,
+                                int32_t num_sms, int32_t *out, int64_t capacity);
+
 /* Bits of a device error word. */
 #define RSWA_DEVERR_TIMEOUT 1
 #define RSWA_DEVERR_BAD_TOKEN 2

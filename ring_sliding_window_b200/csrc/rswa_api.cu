@@ -650,6 +650,21 @@ rswa_status rswa_check_device_error(rswa_state *s, void *stream) {
   return RSWA_OK;
 }
 
+int64_t rswa_debug_prefill_plan(const rswa_config *cfg, const int64_t *prefill_len,
+                                int32_t num_sms, int32_t *out, int64_t capacity) {
+  if (!config_ok(cfg, prefill_len) || num_sms < 1 || capacity < 0 || (capacity > 0 && !out))
+    return -1;
+  const std::vector<int4> blocks = plan_prefill_blocks(cfg, prefill_len, num_sms);
+  const int64_t n = (int64_t)blocks.size();
+  for (int64_t i = 0; i < n && i < capacity; ++i) {
+    out[4 * i] = blocks[(size_t)i].x;
+    out[4 * i + 1] = blocks[(size_t)i].y;
+    out[4 * i + 2] = blocks[(size_t)i].z;
+    out[4 * i + 3] = blocks[(size_t)i].w;
+  }
+  return n;
+}
+
 rswa_status rswa_debug_inject_fault(rswa_state *s, int32_t flags, void *stream) {
   if (!s || (flags & ~(RSWA_FAULT_DROP_DECODE_COPIES | RSWA_FAULT_DROP_PREFILL_LOADS)) != 0)
     return RSWA_EINVAL;

@@ -35,6 +35,7 @@ EXPORTED = (
     "rswa_pool_free", "rswa_pool_stats", "rswa_pool_capacity", "rswa_pool_cache_bytes",
     "rswa_state_create_pooled", "rswa_ngram_topk", "rswa_state_set_rope",
     "rswa_state_set_attention", "rswa_decode_step_partial", "rswa_combine_partials",
+    "rswa_debug_prefill_plan",
 )
 RSWA_ATTN_RING, RSWA_ATTN_STANDARD_SWA = 0, 1
 RSWA_ROPE_NONE, RSWA_ROPE_ABSOLUTE, RSWA_ROPE_SLOT = 0, 1, 2
@@ -113,6 +114,8 @@ lib.rswa_decode_step_noalloc.argtypes = [_cfgp, _i64p, _i64p, _vp, _vp, _vp, _vp
 lib.rswa_decode_step_noalloc.restype = ctypes.c_int
 lib.rswa_debug_inject_fault.argtypes = [_vp, ctypes.c_int32, _vp]
 lib.rswa_debug_inject_fault.restype = ctypes.c_int
+lib.rswa_debug_prefill_plan.argtypes = [_vp, _vp, ctypes.c_int32, _vp, ctypes.c_int64]
+lib.rswa_debug_prefill_plan.restype = ctypes.c_int64
 lib.rswa_last_cuda_error.argtypes = []
 lib.rswa_last_cuda_error.restype = ctypes.c_char_p
 lib.rswa_status_string.argtypes = [ctypes.c_int]
@@ -353,6 +356,22 @@ def rswa_decode_step_noalloc(cfg: rswa_config, prefill_len, n_generated, k_cache
                                         _ptr(k_cache), _ptr(v_cache), _ptr(q), _ptr(k_new),
                                         _ptr(v_new), _ptr(out), _ptr(device_error),
                                         _stream(stream)), "rswa_decode_step_noalloc")
+
+
+def rswa_debug_prefill_plan(batch, num_heads, head_dim, window, dtype, prefill_lens,
+                            num_sms: int):
+    """Test-only: the tensor-core prefill's blocks for this batch on a part
+    with `num_sms` SMs, in launch order, as a list of (b, h, first query tile,
+    query tiles).  Host only."""
+    import numpy as np
+    cfg = make_config(batch, 1, num_heads, head_dim, window, dtype)
+    pl = (ctypes.c_int64 * batch)(*[int(p) for p in prefill_lens])
+    n = lib.rswa_debug_prefill_plan(ctypes.byref(cfg), pl, int(num_sms), None, 0)
+    if n < 0:
+        raise RswaError(RSWA_EINVAL, "rswa_debug_prefill_plan")
+    out = np.zeros((max(int(n), 1), 4), dtype=np.int32)
+    lib.rswa_debug_prefill_plan(ctypes.byref(cfg), pl, int(num_sms), out.ctypes.data, int(n))
+    return [tuple(int(x) for x in row) for row in out[:n]]
 
 
 def rswa_debug_inject_fault(state, flags: int, stream=None) -> None:
